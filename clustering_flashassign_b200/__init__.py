@@ -1,0 +1,190 @@
+"""Python binding of libfk.so (include/fk.h): exact batched Lloyd's K-Means on B200.
+
+Argument marshalling only -- every step of the computation runs in the CUDA
+library.  The functions mirror the C ABI names; they take torch tensors
+(contiguous, row-major), pass their data pointers and sizes, and raise
+``FkError`` when the library returns a status other than FK_OK.  There is no
+fallback: when libfk.so is missing, importing this package raises.
+
+    fk_assign(x, c, ids)                        FlashAssign      (B,N,d),(B,K,d) -> ids (B,N) int32
+    fk_update(x, ids, centers, counts=None)     sort-inverse update, centers (B,K,d) fp32 in/out
+    fk_sort(ids, K, perm, counts=None, offsets=None)
+    fk_lloyd(x, init_centers, max_iter, tol, ids, centers) -> iterations run
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfk.so")
+
+FK_F32, FK_F16, FK_BF16 = 0, 1, 2
+FK_OK, FK_EINVAL, FK_ENOMEM, FK_ECUDA, FK_ETIMEOUT, FK_EUNSUPPORTED = range(6)
+FK_HOST_AUTO, FK_HOST_RESIDENT, FK_HOST_STREAM = 0, 1, 2
+
+DTYPES = {torch.float32: FK_F32, torch.float16: FK_F16, torch.bfloat16: FK_BF16}
+
+EXPORTS = ["fk_assign", "fk_update", "fk_sort", "fk_lloyd", "fk_status_string", "fk_last_error",
+           "fk_device_error", "fk_release", "fk_profile_enable", "fk_profile_read",
+           "fk_launch_count", "fk_version"]
+
+
+class FkError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: status {status} ({detail})")
+        self.status = status
+
+
+class FkShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_longlong), ("K", ctypes.c_int),
+                ("d", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class FkOptions(ctypes.Structure):
+    _fields_ = [("host_mode", ctypes.c_int), ("chunk_points", ctypes.c_longlong),
+                ("verbose", ctypes.c_int)]
+
+
+class FkProfile(ctypes.Structure):
+    _fields_ = [("assign_ms", ctypes.c_double), ("assign_launches", ctypes.c_longlong),
+                ("sort_ms", ctypes.c_double), ("reduce_ms", ctypes.c_double),
+                ("finalize_ms", ctypes.c_double), ("update_calls", ctypes.c_longlong),
+                ("kernel_launches", ctypes.c_longlong)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libfk.so not built at {LIB_PATH}; run python -m clustering_flashassign_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, LL, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
+    sig = {
+        "fk_assign": (I, [P, P, I, LL, I, I, I, P, P]),
+        "fk_update": (I, [P, P, I, LL, I, I, P, P, P, I, P]),
+        "fk_sort": (I, [P, I, LL, I, P, P, P, P]),
+        "fk_lloyd": (I, [ctypes.POINTER(FkShape), P, P, I, F, P, P, P, ctypes.POINTER(I),
+                         ctypes.POINTER(FkOptions)]),
+        "fk_status_string": (ctypes.c_char_p, [I]),
+        "fk_last_error": (ctypes.c_char_p, []),
+        "fk_device_error": (I, [P]),
+        "fk_release": (I, []),
+        "fk_profile_enable": (I, [I]),
+        "fk_profile_read": (I, [ctypes.POINTER(FkProfile), I]),
+        "fk_launch_count": (LL, []),
+        "fk_version": (I, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != FK_OK:
+        detail = lib.fk_last_error().decode(errors="replace") or lib.fk_status_string(status).decode()
+        raise FkError(status, where, detail)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in DTYPES:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    return DTYPES[t.dtype]
+
+
+def fk_assign(x: torch.Tensor, c: torch.Tensor, ids: torch.Tensor, stream=None) -> torch.Tensor:
+    """ids[b,i] = argmin_k ||c_k||^2 - 2 x_i.c_k (lowest k on ties)."""
+    B, N, d = x.shape
+    K = c.shape[1]
+    _check(lib.fk_assign(_ptr(x), _ptr(c), B, N, K, d, _dtype_code(x), _ptr(ids), _stream(stream)),
+           "fk_assign")
+    return ids
+
+
+def fk_update(x: torch.Tensor, ids: torch.Tensor, centers: torch.Tensor, counts=None,
+              max_shift=None, stream=None) -> torch.Tensor:
+    """Sort-inverse update: centers (B,K,d) fp32 in/out, counts (B,K) int32 out."""
+    B, N, d = x.shape
+    K = centers.shape[1]
+    _check(lib.fk_update(_ptr(x), _ptr(ids), B, N, K, d, _ptr(centers), _ptr(counts),
+                         _stream(stream), _dtype_code(x), _ptr(max_shift)), "fk_update")
+    return centers
+
+
+def fk_sort(ids: torch.Tensor, K: int, perm: torch.Tensor, counts=None, offsets=None,
+            stream=None) -> torch.Tensor:
+    """Stable counting sort of ids: perm lists point indices ordered by (id, index)."""
+    B, N = ids.shape
+    _check(lib.fk_sort(_ptr(ids), B, N, K, _ptr(counts), _ptr(offsets), _ptr(perm), _stream(stream)),
+           "fk_sort")
+    return perm
+
+
+def fk_lloyd(x: torch.Tensor, init_centers: torch.Tensor, max_iter: int, tol: float,
+             ids: torch.Tensor, centers: torch.Tensor, stream=None, host_mode: int = FK_HOST_AUTO,
+             chunk_points: int = 0, verbose: bool = False) -> int:
+    """Lloyd loop; x / init / outputs may be device or host tensors. Returns iterations run."""
+    B, N, d = x.shape
+    K = init_centers.shape[1]
+    shape = FkShape(B, N, K, d, _dtype_code(x))
+    opts = FkOptions(host_mode, chunk_points, 1 if verbose else 0)
+    iters = ctypes.c_int(0)
+    _check(lib.fk_lloyd(ctypes.byref(shape), _ptr(x), _ptr(init_centers), int(max_iter), float(tol),
+                        _ptr(ids), _ptr(centers), _stream(stream), ctypes.byref(iters),
+                        ctypes.byref(opts)), "fk_lloyd")
+    return iters.value
+
+
+def fk_device_error(stream=None) -> int:
+    return int(lib.fk_device_error(_stream(stream)))
+
+
+def fk_release() -> None:
+    _check(lib.fk_release(), "fk_release")
+
+
+def fk_profile_enable(on: bool = True) -> None:
+    _check(lib.fk_profile_enable(1 if on else 0), "fk_profile_enable")
+
+
+def fk_profile_read(reset: bool = False) -> dict:
+    p = FkProfile()
+    _check(lib.fk_profile_read(ctypes.byref(p), 1 if reset else 0), "fk_profile_read")
+    return {f: getattr(p, f) for f, _ in FkProfile._fields_}
+
+
+def fk_launch_count() -> int:
+    return int(lib.fk_launch_count())
+
+
+def fk_version() -> int:
+    return int(lib.fk_version())
+
+
+def fk_status_string(status: int) -> str:
+    return lib.fk_status_string(int(status)).decode()
+
+
+def fk_last_error() -> str:
+    return lib.fk_last_error().decode(errors="replace")

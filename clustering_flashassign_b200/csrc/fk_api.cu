@@ -1,0 +1,406 @@
+// The extern "C" surface of libfk (declared in include/fk.h): argument checks,
+// dispatch to the kernels, the Lloyd loop and its streamed (out-of-core) path.
+#include <cstdio>
+#include <cstring>
+
+#include "fk_internal.h"
+
+namespace fk {
+namespace {
+
+enum Loc { LOC_DEVICE, LOC_HOST_PINNED, LOC_HOST_PAGEABLE };
+
+Loc locate(const void *p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return LOC_HOST_PAGEABLE;
+  }
+  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) return LOC_DEVICE;
+  if (at.type == cudaMemoryTypeHost) return LOC_HOST_PINNED;
+  return LOC_HOST_PAGEABLE;
+}
+
+int check_shape(int B, long long N, int K, int d, int dtype) {
+  if (dtype != FK_F32 && dtype != FK_F16 && dtype != FK_BF16)
+    return set_error(FK_EINVAL, "unknown dtype " + std::to_string(dtype));
+  if (B <= 0 || N <= 0 || K <= 0 || d <= 0) return set_error(FK_EINVAL, "B, N, K and d must be positive");
+  if (N > 0x7fffffffLL) return set_error(FK_EINVAL, "N must be below 2^31");
+  if ((long long)K > N) return set_error(FK_EINVAL, "K must not exceed N");
+  if (B > 65535) return set_error(FK_EUNSUPPORTED, "B above 65535");
+  if (K > (1 << 24)) return set_error(FK_EUNSUPPORTED, "K above 2^24");
+  if (dtype != FK_F32 && (d * 2) % 16 != 0)
+    return set_error(FK_EINVAL, "fp16/bf16 rows must be a multiple of 16 bytes (d % 8 == 0)");
+  return FK_OK;
+}
+
+int check_ptr(const void *p, const char *name, bool aligned16) {
+  if (!p) return set_error(FK_EINVAL, std::string(name) + " is NULL");
+  if (aligned16 && (reinterpret_cast<uintptr_t>(p) & 15u))
+    return set_error(FK_EINVAL, std::string(name) + " is not 16-byte aligned");
+  return FK_OK;
+}
+
+int read_device_error(Workspace *ws, cudaStream_t s) {
+  int h = 0;
+  FK_CUDA(cudaMemcpyAsync(&h, ws->err, sizeof(int), cudaMemcpyDeviceToHost, s));
+  FK_CUDA(cudaStreamSynchronize(s));
+  if (h == DEV_OK) return FK_OK;
+  FK_CUDA(cudaMemsetAsync(ws->err, 0, sizeof(int), s));
+  FK_CUDA(cudaStreamSynchronize(s));
+  if (h == DEV_TIMEOUT) return set_error(FK_ETIMEOUT, "a kernel's bounded wait expired");
+  return set_error(FK_EINVAL, "an id outside [0, K) reached the update");
+}
+
+// Sorted keys + perm for `sort_entries` positions and fp32 sums for
+// `sum_rows` centroids of d; the sums stay all-zero between calls (the
+// finalize clears what it reads; a fresh or dirty buffer is cleared here).
+int prepare_update(Workspace *ws, long long sort_entries, long long sum_rows, int d, cudaStream_t s) {
+  FK_TRY(ensure(ws->keys_a, (size_t)sort_entries * sizeof(int32_t)));
+  FK_TRY(ensure(ws->vals_a, (size_t)sort_entries * sizeof(int32_t)));
+  void *old = ws->sums.p;
+  FK_TRY(ensure(ws->sums, (size_t)sum_rows * d * sizeof(float)));
+  if (ws->sums.p != old) ws->sums_dirty = true;
+  if (ws->sums_dirty) {
+    FK_CUDA(cudaMemsetAsync(ws->sums.p, 0, ws->sums.bytes, s));
+    ws->sums_dirty = false;
+  }
+  return FK_OK;
+}
+
+// Steps a2-a5 on device-resident points; ch / cn (nullable) receive the dtype
+// copy and ||c||^2 of the new centroids for the next assign.
+int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long N, int K, int d,
+              int dtype, float *centers, int32_t *counts_out, void *ch, float *cn, long long Kpad,
+              cudaStream_t s) {
+  note_update_call();
+  int32_t *counts = counts_out;
+  if (!counts) {
+    FK_TRY(ensure(ws->counts, (size_t)B * K * sizeof(int32_t)));
+    counts = (int32_t *)ws->counts.p;
+  }
+  FK_TRY(prepare_update(ws, (long long)B * N, (long long)B * K, d, s));
+  FK_CUDA(cudaMemsetAsync(ws->maxshift, 0, sizeof(unsigned), s));
+  int32_t *keys = (int32_t *)ws->keys_a.p, *perm = (int32_t *)ws->vals_a.p;
+  {
+    PhaseTimer t(PH_SORT, s);
+    FK_TRY(run_sort(ws, ids, B, N, K, counts, nullptr, perm, keys, false, s));
+  }
+  int st;
+  {
+    PhaseTimer t(PH_REDUCE, s);
+    st = launch_segreduce(x, dtype, keys, perm, B, N, K, d, (float *)ws->sums.p, s);
+  }
+  if (st != FK_OK) {
+    ws->sums_dirty = true;
+    return st;
+  }
+  {
+    PhaseTimer t(PH_FINALIZE, s);
+    st = launch_finalize((float *)ws->sums.p, counts, centers, ch, cn, dtype, B, K, d, Kpad,
+                         ws->maxshift, s);
+  }
+  if (st != FK_OK) ws->sums_dirty = true;
+  return st;
+}
+
+int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const float *cn, int B,
+                       long long N, int K, int d, int dtype, long long Kpad, int32_t *ids,
+                       cudaStream_t s) {
+  PhaseTimer t(PH_ASSIGN, s);
+  if (dtype == FK_F32) return launch_assign_f32((const float *)x, (const float *)cdt, B, N, K, d, ids, s);
+  return launch_assign_tc(x, cdt, cn, dtype, B, N, K, d, Kpad, ids, ws->err, s);
+}
+
+int read_shift(Workspace *ws, cudaStream_t s, float *out) {
+  FK_CUDA(cudaMemcpyAsync(ws->h_maxshift, ws->maxshift, sizeof(float), cudaMemcpyDeviceToHost, s));
+  FK_CUDA(cudaStreamSynchronize(s));
+  *out = *ws->h_maxshift;
+  return FK_OK;
+}
+
+int ensure_copy_engine(Workspace *ws) {
+  if (!ws->copy_stream) FK_CUDA(cudaStreamCreateWithFlags(&ws->copy_stream, cudaStreamNonBlocking));
+  for (int i = 0; i < 2; ++i) {
+    if (!ws->ready[i]) FK_CUDA(cudaEventCreateWithFlags(&ws->ready[i], cudaEventDisableTiming));
+    if (!ws->freed[i]) FK_CUDA(cudaEventCreateWithFlags(&ws->freed[i], cudaEventDisableTiming));
+  }
+  return FK_OK;
+}
+
+// Out-of-core Lloyd: x stays in host memory and is re-streamed every iteration
+// in chunks, double-buffered so the copy of chunk j+1 overlaps the compute of
+// chunk j ("flash-kmeans and the return of exact K-Means on the GPU", section
+// "Multi-GPU scaling without a NCCL dependency": per-device double-buffered
+// host-to-device plus compute pipeline, and the next iteration's first block
+// prefetched while the current iteration reduces).  Assign, sort and segment
+// reduce run per chunk; counts and sums accumulate over the chunks and the
+// finalize runs once per iteration.
+int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void *init_dev,
+                   int max_iter, float tol, int32_t *ids_dev, float *cen_dev, cudaStream_t s,
+                   int *iters_run, long long chunk, int verbose) {
+  const int B = sh.B, K = sh.K, d = sh.d, dtype = sh.dtype;
+  const long long N = sh.N;
+  const size_t es = esize(dtype);
+  const long long Kpad = kpad_of(K);
+  if (chunk <= 0) chunk = 1LL << 24;
+  if (chunk > N) chunk = N;
+  const long long per_b = (N + chunk - 1) / chunk;
+  FK_TRY(ensure_copy_engine(ws));
+  for (int i = 0; i < 2; ++i) FK_TRY(ensure(ws->chunk[i], (size_t)chunk * d * es));
+  void *ch = nullptr;
+  float *cn = nullptr;
+  if (dtype != FK_F32) {
+    FK_TRY(ensure(ws->ch, (size_t)B * K * d * es));
+    FK_TRY(ensure(ws->cn, (size_t)B * Kpad * sizeof(float)));
+    ch = ws->ch.p;
+    cn = (float *)ws->cn.p;
+  }
+  FK_TRY(ensure(ws->counts, (size_t)B * K * sizeof(int32_t)));
+  int32_t *counts = (int32_t *)ws->counts.p;
+  FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cn, s));
+  FK_TRY(prepare_update(ws, chunk, (long long)B * K, d, s));
+  float *sums = (float *)ws->sums.p;
+  int32_t *keys = (int32_t *)ws->keys_a.p, *perm = (int32_t *)ws->vals_a.p;
+  long long job = 0;
+  int it = 0;
+  for (it = 0; it < max_iter; ++it) {
+    note_update_call();
+    FK_CUDA(cudaMemsetAsync(counts, 0, (size_t)B * K * sizeof(int32_t), s));
+    FK_CUDA(cudaMemsetAsync(ws->maxshift, 0, sizeof(unsigned), s));
+    for (int b = 0; b < B; ++b) {
+      for (long long ci = 0; ci < per_b; ++ci, ++job) {
+        const int buf = (int)(job & 1);
+        const long long n0 = ci * chunk;
+        const long long nc = (n0 + chunk <= N) ? chunk : N - n0;
+        void *xb = ws->chunk[buf].p;
+        FK_CUDA(cudaStreamWaitEvent(ws->copy_stream, ws->freed[buf], 0));
+        FK_CUDA(cudaMemcpyAsync(xb, xh + ((size_t)b * N + n0) * d * es, (size_t)nc * d * es,
+                                cudaMemcpyHostToDevice, ws->copy_stream));
+        FK_CUDA(cudaEventRecord(ws->ready[buf], ws->copy_stream));
+        FK_CUDA(cudaStreamWaitEvent(s, ws->ready[buf], 0));
+        int32_t *idc = ids_dev + (size_t)b * N + n0;
+        const void *cb = dtype == FK_F32 ? (const void *)(cen_dev + (size_t)b * K * d)
+                                         : (const void *)((const char *)ch + (size_t)b * K * d * es);
+        FK_TRY(do_assign_resident(ws, xb, cb, cn ? cn + (size_t)b * Kpad : nullptr, 1, nc, K, d, dtype,
+                                  Kpad, idc, s));
+        {
+          PhaseTimer t(PH_SORT, s);
+          FK_TRY(run_sort(ws, idc, 1, nc, K, counts + (size_t)b * K, nullptr, perm, keys, true, s));
+        }
+        {
+          PhaseTimer t(PH_REDUCE, s);
+          int st = launch_segreduce(xb, dtype, keys, perm, 1, nc, K, d, sums + (size_t)b * K * d, s);
+          if (st != FK_OK) {
+            ws->sums_dirty = true;
+            return st;
+          }
+        }
+        FK_CUDA(cudaEventRecord(ws->freed[buf], s));
+      }
+    }
+    {
+      PhaseTimer t(PH_FINALIZE, s);
+      int st = launch_finalize(sums, counts, cen_dev, ch, cn, dtype, B, K, d, Kpad, ws->maxshift, s);
+      if (st != FK_OK) {
+        ws->sums_dirty = true;
+        return st;
+      }
+    }
+    if (tol > 0.f || verbose) {
+      float ms = 0.f;
+      FK_TRY(read_shift(ws, s, &ms));
+      if (verbose) fprintf(stderr, "fk_lloyd(streamed) iter %d max_shift %.6g\n", it + 1, ms);
+      if (tol > 0.f && ms < tol) {
+        ++it;
+        break;
+      }
+    }
+  }
+  *iters_run = it;
+  return FK_OK;
+}
+
+}  // namespace
+}  // namespace fk
+
+using namespace fk;
+
+extern "C" {
+
+int fk_assign(const void *x, const void *c, int B, long long N, int K, int d, int dtype,
+              int32_t *ids, fk_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FK_TRY(check_shape(B, N, K, d, dtype));
+  const bool tc = dtype != FK_F32;
+  FK_TRY(check_ptr(x, "x", tc));
+  FK_TRY(check_ptr(c, "c", tc));
+  FK_TRY(check_ptr(ids, "ids", false));
+  Workspace *ws;
+  FK_TRY(workspace_for(s, &ws));
+  const long long Kpad = kpad_of(K);
+  float *cn = nullptr;
+  if (tc) {
+    FK_TRY(ensure(ws->cn, (size_t)B * Kpad * sizeof(float)));
+    cn = (float *)ws->cn.p;
+    FK_TRY(launch_prep_cn(c, dtype, B, K, d, Kpad, cn, s));
+  }
+  return do_assign_resident(ws, x, c, cn, B, N, K, d, dtype, Kpad, ids, s);
+}
+
+int fk_update(const void *x, const int32_t *ids, int B, long long N, int K, int d, float *centers,
+              int32_t *counts, fk_stream_t stream, int dtype, float *max_shift) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FK_TRY(check_shape(B, N, K, d, dtype));
+  FK_TRY(check_ptr(x, "x", true));
+  FK_TRY(check_ptr(ids, "ids", false));
+  FK_TRY(check_ptr(centers, "centers", true));
+  Workspace *ws;
+  FK_TRY(workspace_for(s, &ws));
+  FK_TRY(do_update(ws, x, ids, B, N, K, d, dtype, centers, counts, nullptr, nullptr, kpad_of(K), s));
+  if (max_shift)
+    FK_CUDA(cudaMemcpyAsync(max_shift, ws->maxshift, sizeof(float), cudaMemcpyDeviceToDevice, s));
+  return FK_OK;
+}
+
+int fk_sort(const int32_t *ids, int B, long long N, int K, int32_t *counts, int32_t *offsets,
+            int32_t *perm, fk_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FK_TRY(check_shape(B, N, K, 8, FK_F32));
+  FK_TRY(check_ptr(ids, "ids", false));
+  FK_TRY(check_ptr(perm, "perm", false));
+  Workspace *ws;
+  FK_TRY(workspace_for(s, &ws));
+  PhaseTimer t(PH_SORT, s);
+  return run_sort(ws, ids, B, N, K, counts, offsets, perm, nullptr, false, s);
+}
+
+int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int max_iter,
+             float tol, int32_t *ids, float *centers, fk_stream_t stream, int *iters_run,
+             const fk_options *opts) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!shape) return set_error(FK_EINVAL, "shape is NULL");
+  const fk_shape sh = *shape;
+  FK_TRY(check_shape(sh.B, sh.N, sh.K, sh.d, sh.dtype));
+  FK_TRY(check_ptr(x, "x", true));
+  FK_TRY(check_ptr(init_centers, "init_centers", false));
+  FK_TRY(check_ptr(ids, "ids", false));
+  FK_TRY(check_ptr(centers, "centers", true));
+  if (max_iter < 0) return set_error(FK_EINVAL, "max_iter must be >= 0");
+  fk_options o{FK_HOST_AUTO, 0, 0};
+  if (opts) o = *opts;
+  const int B = sh.B, K = sh.K, d = sh.d, dtype = sh.dtype;
+  const long long N = sh.N;
+  const size_t es = esize(dtype);
+  const size_t xbytes = (size_t)B * N * d * es;
+  const size_t cbytes = (size_t)B * K * d * es;
+  const long long Kpad = kpad_of(K);
+  Workspace *ws;
+  FK_TRY(workspace_for(s, &ws));
+
+  const Loc lx = locate(x), li = locate(init_centers), lids = locate(ids), lc = locate(centers);
+  const void *init_dev = init_centers;
+  if (li != LOC_DEVICE) {
+    FK_TRY(ensure(ws->init_dev, cbytes));
+    FK_CUDA(cudaMemcpyAsync(ws->init_dev.p, init_centers, cbytes, cudaMemcpyHostToDevice, s));
+    init_dev = ws->init_dev.p;
+  }
+  int32_t *ids_dev = ids;
+  if (lids != LOC_DEVICE) {
+    FK_TRY(ensure(ws->ids_dev, (size_t)B * N * sizeof(int32_t)));
+    ids_dev = (int32_t *)ws->ids_dev.p;
+  }
+  float *cen_dev = centers;
+  if (lc != LOC_DEVICE) {
+    FK_TRY(ensure(ws->centers_dev, (size_t)B * K * d * sizeof(float)));
+    cen_dev = (float *)ws->centers_dev.p;
+  }
+
+  int iters = 0;
+  bool streamed = false;
+  const void *xdev = x;
+  if (lx != LOC_DEVICE) {
+    int mode = o.host_mode;
+    if (mode == FK_HOST_AUTO) {
+      size_t fr = 0, tot = 0;
+      FK_CUDA(cudaMemGetInfo(&fr, &tot));
+      mode = (xbytes + (size_t)(2ull << 30) < fr) ? FK_HOST_RESIDENT : FK_HOST_STREAM;
+    }
+    if (mode == FK_HOST_STREAM) {
+      streamed = true;
+      FK_TRY(lloyd_streamed(ws, sh, (const char *)x, init_dev, max_iter, tol, ids_dev, cen_dev, s,
+                            &iters, o.chunk_points, o.verbose));
+    } else {
+      FK_TRY(ensure(ws->xres, xbytes));
+      FK_CUDA(cudaMemcpyAsync(ws->xres.p, x, xbytes, cudaMemcpyHostToDevice, s));
+      xdev = ws->xres.p;
+    }
+  }
+  if (!streamed) {
+    void *ch = nullptr;
+    float *cn = nullptr;
+    if (dtype != FK_F32) {
+      FK_TRY(ensure(ws->ch, cbytes));
+      FK_TRY(ensure(ws->cn, (size_t)B * Kpad * sizeof(float)));
+      ch = ws->ch.p;
+      cn = (float *)ws->cn.p;
+    }
+    FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cn, s));
+    const void *cassign = dtype == FK_F32 ? (const void *)cen_dev : ch;
+    for (int it = 0; it < max_iter; ++it) {
+      FK_TRY(do_assign_resident(ws, xdev, cassign, cn, B, N, K, d, dtype, Kpad, ids_dev, s));
+      FK_TRY(do_update(ws, xdev, ids_dev, B, N, K, d, dtype, cen_dev, nullptr, ch, cn, Kpad, s));
+      iters = it + 1;
+      if (tol > 0.f || o.verbose) {
+        float ms = 0.f;
+        FK_TRY(read_shift(ws, s, &ms));
+        if (o.verbose) fprintf(stderr, "fk_lloyd iter %d max_shift %.6g\n", it + 1, ms);
+        if (tol > 0.f && ms < tol) break;
+      }
+    }
+  }
+  if (ids_dev != ids)
+    FK_CUDA(cudaMemcpyAsync(ids, ids_dev, (size_t)B * N * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  if (cen_dev != centers)
+    FK_CUDA(cudaMemcpyAsync(centers, cen_dev, (size_t)B * K * d * sizeof(float), cudaMemcpyDeviceToHost, s));
+  FK_CUDA(cudaStreamSynchronize(s));
+  FK_TRY(read_device_error(ws, s));
+  if (iters_run) *iters_run = iters;
+  return FK_OK;
+}
+
+const char *fk_status_string(int status) {
+  switch (status) {
+    case FK_OK: return "ok";
+    case FK_EINVAL: return "invalid argument";
+    case FK_ENOMEM: return "out of device memory";
+    case FK_ECUDA: return "CUDA runtime error";
+    case FK_ETIMEOUT: return "kernel wait timed out";
+    case FK_EUNSUPPORTED: return "unsupported shape";
+    default: return "unknown status";
+  }
+}
+
+const char *fk_last_error(void) { return last_error(); }
+
+int fk_device_error(fk_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Workspace *ws;
+  FK_TRY(workspace_for(s, &ws));
+  return read_device_error(ws, s);
+}
+
+int fk_release(void) {
+  FK_CUDA(cudaDeviceSynchronize());
+  return release_device_workspaces();
+}
+
+int fk_profile_enable(int on) { return profile_enable(on); }
+
+int fk_profile_read(fk_profile *out, int reset) { return profile_read(out, reset); }
+
+long long fk_launch_count(void) { return launch_count(); }
+
+int fk_version(void) { return 100; }
+
+}  // extern "C"

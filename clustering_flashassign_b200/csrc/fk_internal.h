@@ -1,0 +1,118 @@
+// Internal declarations shared by the libfk CUDA sources.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <string>
+
+#include "../../include/fk.h"
+
+namespace fk {
+
+// Device error word values (written by kernels, read by fk_device_error).
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_ID = 2 };
+
+// Bounded waits inside kernels give up after this many nanoseconds.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// Tile geometry of the tensor-core assign.
+constexpr int kTileM = 128;   // points per tile (MMA M)
+constexpr int kChunkN = 256;  // centroids per chunk (MMA N)
+constexpr int kBlockK = 64;   // elements of d per K-block (128-byte rows for 16-bit types)
+
+inline long long kpad_of(int K) { return ((long long)K + kChunkN - 1) / kChunkN * kChunkN; }
+
+// Counting-sort geometry.
+constexpr int kSortWarps = 8;
+constexpr int kSortRounds = 16;
+constexpr int kSortTile = kSortWarps * kSortRounds * 32;  // 4096 points per CTA
+constexpr int kMaxDigitBits = 12;                         // 4096 bins per pass at most
+
+// Segment-reduce geometry.
+constexpr int kPiece = 64;  // sorted positions per segment piece
+
+struct DevBuf {
+  void *p = nullptr;
+  size_t bytes = 0;
+};
+
+// Per (device, stream) scratch.  Grow-only; freed by fk_release().
+struct Workspace {
+  int device = -1;
+  cudaStream_t stream = nullptr;
+  int *err = nullptr;             // device error word
+  unsigned *maxshift = nullptr;   // device, float bits (non-negative floats order as uints)
+  float *h_maxshift = nullptr;    // pinned host mirror
+  DevBuf cn, ch, sums, counts, offsets, table, keys_a, vals_a, keys_b, vals_b;
+  DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2];
+  bool sums_dirty = true;
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
+};
+
+// Status plumbing (thread-local last-error text).
+int set_error(int status, const std::string &msg);
+int cuda_status(cudaError_t e, const char *what);
+#define FK_CUDA(call)                                        \
+  do {                                                       \
+    cudaError_t e_ = (call);                                 \
+    if (e_ != cudaSuccess) return ::fk::cuda_status(e_, #call); \
+  } while (0)
+#define FK_TRY(expr)              \
+  do {                            \
+    int s_ = (expr);              \
+    if (s_ != FK_OK) return s_;   \
+  } while (0)
+
+int ensure(DevBuf &b, size_t bytes);               // grow-only device buffer
+int workspace_for(cudaStream_t s, Workspace **out);
+
+// Launch accounting and event timing.
+void count_launch(int n = 1);
+enum Phase { PH_ASSIGN = 0, PH_SORT = 1, PH_REDUCE = 2, PH_FINALIZE = 3 };
+struct PhaseTimer {
+  cudaEvent_t a = nullptr, b = nullptr;
+  int phase;
+  cudaStream_t s;
+  PhaseTimer(int ph, cudaStream_t st);
+  ~PhaseTimer();
+};
+void note_update_call();
+int release_device_workspaces();
+long long launch_count();
+int profile_enable(int on);
+int profile_read(fk_profile *out, int reset);
+const char *last_error();
+
+size_t esize(int dtype);
+int num_sms();
+
+// ---- kernels (launchers return fk_status) ----
+// centroid preparation: cn[b, k] = ||c[b,k]||^2 (fp32), +inf on [K, Kpad).
+int launch_prep_cn(const void *c, int dtype, int B, int K, int d, long long Kpad, float *cn,
+                   cudaStream_t s);
+// init for fk_lloyd: master = float(init), ch = init (16-bit dtypes), cn.
+int launch_init_centers(const void *init, int dtype, int B, int K, int d, long long Kpad,
+                        float *master, void *ch, float *cn, cudaStream_t s);
+// finalize: new = sums / count or old; shift max; master, ch, cn; zero sums.
+int launch_finalize(float *sums, const int32_t *counts, float *centers, void *ch, float *cn,
+                    int dtype, int B, int K, int d, long long Kpad, unsigned *maxshift,
+                    cudaStream_t s);
+
+int launch_assign_f32(const float *x, const float *c, int B, long long N, int K, int d,
+                      int32_t *ids, cudaStream_t s);
+int launch_assign_tc(const void *x, const void *ch, const float *cn, int dtype, int B, long long N,
+                     int K, int d, long long Kpad, int32_t *ids, int *err, cudaStream_t s);
+
+// counting sort: counts / offsets optional; keys_out + perm always written.
+// accumulate_counts: add into counts instead of overwriting.
+int run_sort(Workspace *ws, const int32_t *ids, int B, long long N, int K, int32_t *counts,
+             int32_t *offsets, int32_t *perm, int32_t *keys_out, bool accumulate_counts,
+             cudaStream_t s);
+
+int launch_segreduce(const void *x, int dtype, const int32_t *skeys, const int32_t *perm, int B,
+                     long long N, int K, int d, float *sums, cudaStream_t s);
+
+}  // namespace fk

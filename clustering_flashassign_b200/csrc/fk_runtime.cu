@@ -1,0 +1,206 @@
+// Runtime pieces of libfk: status text, per-(device, stream) workspaces,
+// launch accounting and event-based phase timing.
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "fk_internal.h"
+
+namespace fk {
+
+namespace {
+thread_local std::string g_last_error;
+std::mutex g_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace *> g_ws;
+std::atomic<long long> g_launches{0};
+
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+struct Pending {
+  cudaEvent_t a, b;
+  int phase;
+};
+std::vector<Pending> g_pending;
+double g_ms[4] = {0, 0, 0, 0};
+long long g_assign_launches = 0, g_update_calls = 0, g_prof_launches = 0;
+}  // namespace
+
+int set_error(int status, const std::string &msg) {
+  g_last_error = msg;
+  return status;
+}
+
+int cuda_status(cudaError_t e, const char *what) {
+  g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+  if (e == cudaErrorMemoryAllocation) return FK_ENOMEM;
+  return FK_ECUDA;
+}
+
+int ensure(DevBuf &b, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  if (b.bytes >= bytes) return FK_OK;
+  if (b.p) {
+    FK_CUDA(cudaFree(b.p));
+    b.p = nullptr;
+    b.bytes = 0;
+  }
+  size_t want = bytes + bytes / 8;  // headroom for small growth
+  cudaError_t e = cudaMalloc(&b.p, want);
+  if (e != cudaSuccess) {
+    b.p = nullptr;
+    e = cudaMalloc(&b.p, bytes);
+    if (e != cudaSuccess) {
+      b.p = nullptr;
+      (void)cudaGetLastError();
+      return set_error(FK_ENOMEM, "device workspace allocation of " + std::to_string(bytes) + " bytes failed");
+    }
+    want = bytes;
+  }
+  b.bytes = want;
+  return FK_OK;
+}
+
+int workspace_for(cudaStream_t s, Workspace **out) {
+  int dev = 0;
+  FK_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto key = std::make_pair(dev, s);
+  auto it = g_ws.find(key);
+  if (it != g_ws.end()) {
+    *out = it->second;
+    return FK_OK;
+  }
+  Workspace *ws = new Workspace();
+  ws->device = dev;
+  ws->stream = s;
+  cudaError_t e = cudaMalloc(&ws->err, 16);
+  if (e == cudaSuccess) e = cudaMemset(ws->err, 0, 16);
+  if (e == cudaSuccess) ws->maxshift = reinterpret_cast<unsigned *>(ws->err + 1);
+  if (e == cudaSuccess) e = cudaMallocHost(&ws->h_maxshift, 16);
+  if (e != cudaSuccess) {
+    if (ws->err) cudaFree(ws->err);
+    delete ws;
+    return cuda_status(e, "workspace setup");
+  }
+  g_ws[key] = ws;
+  *out = ws;
+  return FK_OK;
+}
+
+static void free_buf(DevBuf &b) {
+  if (b.p) cudaFree(b.p);
+  b.p = nullptr;
+  b.bytes = 0;
+}
+
+int release_device_workspaces() {
+  int dev = 0;
+  FK_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto it = g_ws.begin(); it != g_ws.end();) {
+    if (it->first.first != dev) {
+      ++it;
+      continue;
+    }
+    Workspace *ws = it->second;
+    DevBuf *bufs[] = {&ws->cn, &ws->ch, &ws->sums, &ws->counts, &ws->offsets, &ws->table,
+                      &ws->keys_a, &ws->vals_a, &ws->keys_b, &ws->vals_b, &ws->xres,
+                      &ws->init_dev, &ws->ids_dev, &ws->centers_dev, &ws->chunk[0], &ws->chunk[1]};
+    for (DevBuf *b : bufs) free_buf(*b);
+    if (ws->err) cudaFree(ws->err);
+    if (ws->h_maxshift) cudaFreeHost(ws->h_maxshift);
+    if (ws->copy_stream) cudaStreamDestroy(ws->copy_stream);
+    for (int i = 0; i < 2; ++i) {
+      if (ws->ready[i]) cudaEventDestroy(ws->ready[i]);
+      if (ws->freed[i]) cudaEventDestroy(ws->freed[i]);
+    }
+    delete ws;
+    it = g_ws.erase(it);
+  }
+  return FK_OK;
+}
+
+void count_launch(int n) {
+  g_launches.fetch_add(n, std::memory_order_relaxed);
+  if (g_prof_on) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_launches += n;
+  }
+}
+
+long long launch_count() { return g_launches.load(); }
+
+PhaseTimer::PhaseTimer(int ph, cudaStream_t st) : phase(ph), s(st) {
+  if (!g_prof_on) return;
+  if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) {
+    a = b = nullptr;
+    return;
+  }
+  cudaEventRecord(a, s);
+}
+
+PhaseTimer::~PhaseTimer() {
+  if (!a) return;
+  cudaEventRecord(b, s);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_pending.push_back({a, b, phase});
+  if (phase == PH_ASSIGN) ++g_assign_launches;
+}
+
+void note_update_call() {
+  if (!g_prof_on) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  ++g_update_calls;
+}
+
+int profile_enable(int on) {
+  g_prof_on = on != 0;
+  return FK_OK;
+}
+
+int profile_read(fk_profile *out, int reset) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto &p : g_pending) {
+    float ms = 0.f;
+    cudaEventSynchronize(p.b);
+    if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) g_ms[p.phase] += ms;
+    cudaEventDestroy(p.a);
+    cudaEventDestroy(p.b);
+  }
+  g_pending.clear();
+  if (out) {
+    out->assign_ms = g_ms[PH_ASSIGN];
+    out->sort_ms = g_ms[PH_SORT];
+    out->reduce_ms = g_ms[PH_REDUCE];
+    out->finalize_ms = g_ms[PH_FINALIZE];
+    out->assign_launches = g_assign_launches;
+    out->update_calls = g_update_calls;
+    out->kernel_launches = g_prof_launches;
+  }
+  if (reset) {
+    for (double &v : g_ms) v = 0;
+    g_assign_launches = g_update_calls = g_prof_launches = 0;
+  }
+  return FK_OK;
+}
+
+size_t esize(int dtype) { return dtype == FK_F32 ? 4 : 2; }
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+const char *last_error() { return g_last_error.c_str(); }
+
+}  // namespace fk

@@ -1,0 +1,211 @@
+/*
+ * fk.h -- C ABI of libfk.so: exact batched Lloyd's K-Means on one NVIDIA
+ * B200 (sm_100a).
+ *
+ * The library implements the two kernel-level ideas of flash-kmeans:
+ *   - FlashAssign: the point-to-centroid distance is fused with a running
+ *     argmin, so the (B, N, K) distance matrix never exists
+ *     ("Flash-KMeans: Fast and Memory-Efficient Exact K-Means", Abstract;
+ *     "flash-kmeans and the return of exact K-Means on the GPU", section
+ *     "The point of the kernel is that the distance matrix never exists").
+ *   - Sort-inverse update: the assignment vector is sorted by cluster id
+ *     (a stable counting sort here), each contiguous segment is reduced on
+ *     chip and flushed with one atomic add per segment piece
+ *     ("Flash-KMeans: IO感知的精确K-Means", section "它攻克的兩大瓶頸").
+ * plus the chunked host-to-device stream overlap for point sets held in
+ * pinned host memory (same Abstract; "flash-kmeans and the return of exact
+ * K-Means on the GPU", section "Multi-GPU scaling without a NCCL
+ * dependency", the double-buffered host-to-device pipeline).
+ *
+ * Conventions shared by every entry point
+ *   - Layouts are dense row-major: points x (B, N, d), centroids (B, K, d),
+ *     ids (B, N), counts / offsets (B, K), perm (B, N).  d is contiguous.
+ *   - dtype is one of FK_F32, FK_F16, FK_BF16 and describes x and any
+ *     centroid tensor passed "in x's dtype".  Accumulation is fp32.
+ *   - Pointers are device pointers unless stated otherwise.  The caller owns
+ *     every buffer it passes.  The library keeps its own scratch (workspace)
+ *     per (device, stream), allocated on first use and grown as needed;
+ *     fk_release() frees it.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default
+ *     stream) unless stated otherwise.
+ *   - Every call returns an fk_status.  Nothing throws across the ABI.
+ *     FK_EINVAL: a size <= 0, K > N, N or K beyond 2^31-1, a null pointer,
+ *     an unknown dtype, or (fp16 / bf16) d*2 not a multiple of 16 bytes or a
+ *     pointer not 16-byte aligned.  FK_EUNSUPPORTED: a shape beyond the
+ *     limits stated per call.  FK_ECUDA: a CUDA runtime error (see
+ *     fk_last_error()).  FK_ETIMEOUT: a kernel's bounded wait expired (the
+ *     kernel recorded it in the device error word and returned; see
+ *     fk_device_error()).
+ *   - Ties in the argmin go to the lowest centroid index.  An empty cluster
+ *     keeps its previous centroid.
+ */
+#ifndef FK_H
+#define FK_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *fk_stream_t; /* identical to cudaStream_t */
+
+typedef enum { FK_F32 = 0, FK_F16 = 1, FK_BF16 = 2 } fk_dtype;
+
+typedef enum {
+  FK_OK = 0,
+  FK_EINVAL = 1,
+  FK_ENOMEM = 2,
+  FK_ECUDA = 3,
+  FK_ETIMEOUT = 4,
+  FK_EUNSUPPORTED = 5
+} fk_status;
+
+/* Problem shape for fk_lloyd. */
+typedef struct {
+  int B;       /* independent problems (batches) */
+  long long N; /* points per batch, 1 <= N <= 2^31-1 */
+  int K;       /* centroids per batch, 1 <= K <= min(N, 2^24) */
+  int d;       /* dimensions */
+  int dtype;   /* fk_dtype of x and init_centers */
+} fk_shape;
+
+/* Where fk_lloyd keeps points that arrive in host memory. */
+typedef enum {
+  FK_HOST_AUTO = 0,     /* resident copy when it fits in free device memory, else streamed */
+  FK_HOST_RESIDENT = 1, /* copy x to the device once, iterate there */
+  FK_HOST_STREAM = 2    /* re-stream x in chunks every iteration (out-of-core path) */
+} fk_host_mode;
+
+typedef struct {
+  int host_mode;          /* fk_host_mode; used only when x is host memory */
+  long long chunk_points; /* streamed path: points per chunk; 0 = 2^24 */
+  int verbose;            /* 1: one line per iteration on stderr */
+} fk_options;
+
+/*
+ * fk_assign -- FlashAssign (step a1).
+ * ids[b,i] = argmin_k ( ||c[b,k]||^2 - 2 x[b,i].c[b,k] ), fp32 accumulation,
+ * lowest k on ties; the (B, N, K) distance matrix is never written.
+ * Passage: "Flash-KMeans: Fast and Memory-Efficient Exact K-Means", Abstract
+ * (FlashAssign fuses distance computation with an online argmin);
+ * "flash-kmeans and the return of exact K-Means on the GPU", section "The
+ * point of the kernel is that the distance matrix never exists" (point tiles
+ * and centroid chunks streamed on chip).
+ *   x    (B, N, d) in dtype, device.  c (B, K, d) in dtype, device.
+ *   ids  (B, N) int32 out, device.
+ * fp16 / bf16 run on tcgen05 tensor cores (TMA-fed tiles, TMEM accumulators);
+ * fp32 runs on CUDA cores and evaluates sum_j (x_j - c_j)^2 directly (same
+ * argmin, no cancellation).
+ */
+int fk_assign(const void *x, const void *c, int B, long long N, int K, int d, int dtype,
+              int32_t *ids, fk_stream_t stream);
+
+/*
+ * fk_update -- sort-inverse centroid update (steps a2-a5).
+ * counts[b,k] = #{i : ids[b,i] = k};  centers[b,k] = mean of its points in
+ * fp32, or unchanged when counts[b,k] = 0.  The points are gathered in
+ * sorted order without being permuted; each segment piece is reduced on chip
+ * and flushed with one vector atomic add.
+ * Passage: "Flash-KMeans: IO感知的精确K-Means", section "它攻克的兩大瓶頸"
+ * (argsort of the assignment vector, contiguous segments, one atomic add per
+ * segment); "Flash-KMeans: Fast and Memory-Efficient Exact K-Means",
+ * Abstract (explicit inverse mapping).
+ *   x        (B, N, d) in dtype, device.  ids (B, N) int32 in [0, K), device.
+ *   centers  (B, K, d) fp32, device, in: previous centroids, out: new ones.
+ *   counts   (B, K) int32 out, device; may be NULL.
+ *   max_shift  nullable device float: max over b,k of ||new - old||_2.
+ * ids outside [0, K) are a caller error: they are counted nowhere and the
+ * device error word records FK_EINVAL (read it with fk_device_error()).
+ */
+int fk_update(const void *x, const int32_t *ids, int B, long long N, int K, int d,
+              float *centers, int32_t *counts, fk_stream_t stream, int dtype, float *max_shift);
+
+/*
+ * fk_sort -- the stable counting sort inside fk_update (steps a2-a4),
+ * exposed on its own.
+ * counts[b,k] = #{i : ids[b,i] = k};  offsets[b,k] = sum_{k'<k} counts[b,k'];
+ * perm[b, offsets[b,id] + r] = i where r counts the earlier points of the
+ * same batch with the same id (so perm lists point indices ordered by
+ * (id, index)).
+ * Passage: "Flash-KMeans: IO感知的精确K-Means", section "它攻克的兩大瓶頸"
+ * (sort the assignment vector by cluster id into contiguous segments).
+ *   ids (B, N) int32 in [0, K), device.  counts, offsets (B, K) int32 out,
+ *   device, each may be NULL.  perm (B, N) int32 out, device.
+ */
+int fk_sort(const int32_t *ids, int B, long long N, int K, int32_t *counts, int32_t *offsets,
+            int32_t *perm, fk_stream_t stream);
+
+/*
+ * fk_lloyd -- the Lloyd loop (steps a1-a7).
+ * Initial centroids are init_centers (the caller picks them, e.g. a seeded
+ * index set of points).  Each iteration assigns every point, then updates
+ * the centroids; after iteration t the loop stops when the max centroid
+ * shift is below tol (strict: tol <= 0 always runs max_iter iterations).
+ * On return ids holds the last assignment and centers the centroids of the
+ * last update.  The fp32 centroids are rounded to dtype (nearest even)
+ * before each assign.
+ * Passage: "flash-kmeans and the return of exact K-Means on the GPU",
+ * section "Exact K-Means, with the assignment step written in Triton"
+ * (batch_kmeans_Euclid(x, n_clusters, tol, verbose) returning ids and
+ * centers); "Flash-KMeans: IO感知的精确K-Means", section "什么是 Flash-KMeans"
+ * (one Lloyd iteration = assign + update, exact).
+ *   x             (B, N, d) in dtype: device memory, or host memory
+ *                 (pinned for overlap); see fk_options.host_mode.
+ *   init_centers  (B, K, d) in dtype, device or host.
+ *   ids           (B, N) int32 out, device or host.
+ *   centers       (B, K, d) fp32 out, device or host.
+ *   iters_run     nullable host int: iterations executed.
+ *   opts          nullable: defaults {FK_HOST_AUTO, 2^24, 0}.
+ * fk_lloyd synchronizes `stream` before returning and reports any device
+ * error word.  Streamed mode keeps two chunk buffers on the device and
+ * overlaps the copy of the next chunk with the compute of this one.
+ */
+int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int max_iter,
+             float tol, int32_t *ids, float *centers, fk_stream_t stream, int *iters_run,
+             const fk_options *opts);
+
+/* Static text for a status code. */
+const char *fk_status_string(int status);
+
+/* Text of the last FK_ECUDA / FK_EINVAL detail recorded by this thread. */
+const char *fk_last_error(void);
+
+/*
+ * Synchronizes `stream`, reads and clears the device error word of its
+ * workspace.  Returns FK_OK, FK_ETIMEOUT (a bounded wait in a kernel gave
+ * up) or FK_EINVAL (an id outside [0, K) reached fk_update / fk_sort).
+ */
+int fk_device_error(fk_stream_t stream);
+
+/* Frees every workspace of the current device (no call may be in flight). */
+int fk_release(void);
+
+/* Per-phase device time, measured with CUDA events on the launching stream. */
+typedef struct {
+  double assign_ms;   /* FlashAssign / fp32 assign kernels */
+  long long assign_launches;
+  double sort_ms;     /* counting sort kernels of the update */
+  double reduce_ms;   /* segment-reduce kernel */
+  double finalize_ms; /* divide / shift / dtype copy kernel */
+  long long update_calls;
+  long long kernel_launches; /* every kernel this library launched while enabled */
+} fk_profile;
+
+/* Turns event timing on (1) or off (0).  Off by default. */
+int fk_profile_enable(int on);
+
+/* Synchronizes the recorded events, fills *out, and clears the totals if reset != 0. */
+int fk_profile_read(fk_profile *out, int reset);
+
+/* Count of kernel launches issued by this library since load. */
+long long fk_launch_count(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int fk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FK_H */

@@ -80,6 +80,13 @@ static double half_to_double(uint16_t h) {
   return sign ? -v : v;
 }
 
+/* All 65536 binary16 values, widened once by half_to_double at load time. */
+static double g_half_table[65536];
+
+__attribute__((constructor)) static void build_half_table(void) {
+  for (uint32_t h = 0; h < 65536u; ++h) g_half_table[h] = half_to_double((uint16_t)h);
+}
+
 static double bf16_to_double(uint16_t h) {
   uint32_t u = (uint32_t)h << 16;
   float f;
@@ -89,7 +96,7 @@ static double bf16_to_double(uint16_t h) {
 
 static inline double load_x(const void *x, int dtype, size_t i) {
   if (dtype == OR_F32) return (double)((const float *)x)[i];
-  if (dtype == OR_F16) return half_to_double(((const uint16_t *)x)[i]);
+  if (dtype == OR_F16) return g_half_table[((const uint16_t *)x)[i]];
   return bf16_to_double(((const uint16_t *)x)[i]);
 }
 
@@ -241,16 +248,24 @@ int or_update(const void *x, int dtype, const int32_t *ids, int B, long long N, 
               const double *old_c, double *new_c, int64_t *counts, double *shift,
               double *maxshift) {
   if (!x || !ids || !old_c || !new_c || B <= 0 || N <= 0 || K <= 0 || d <= 0) return 1;
-  double *sum = (double *)calloc((size_t)K * d, sizeof(double));
-  int64_t *cnt = (int64_t *)calloc((size_t)K, sizeof(int64_t));
-  if (!sum || !cnt) { free(sum); free(cnt); return 3; }
+  for (size_t i = 0; i < (size_t)B * (size_t)N; ++i)
+    if (ids[i] < 0 || ids[i] >= K) return 2;
   double mx = 0.0;
+  int rc = 0;
+  /* batches are independent problems; each thread owns whole batches */
+#pragma omp parallel for schedule(dynamic, 1) reduction(max : mx)
   for (int b = 0; b < B; ++b) {
-    memset(sum, 0, sizeof(double) * (size_t)K * d);
-    memset(cnt, 0, sizeof(int64_t) * (size_t)K);
+    double *sum = (double *)calloc((size_t)K * d, sizeof(double));
+    int64_t *cnt = (int64_t *)calloc((size_t)K, sizeof(int64_t));
+    if (!sum || !cnt) {
+      free(sum);
+      free(cnt);
+#pragma omp atomic write
+      rc = 3;
+      continue;
+    }
     for (long long i = 0; i < N; ++i) {
       int32_t k = ids[(size_t)b * N + i];
-      if (k < 0 || k >= K) { free(sum); free(cnt); return 2; }
       cnt[k]++;
       size_t xrow = ((size_t)b * (size_t)N + (size_t)i) * (size_t)d;
       double *s = sum + (size_t)k * d;
@@ -277,11 +292,11 @@ int or_update(const void *x, int dtype, const int32_t *ids, int B, long long N, 
       if (sh > mx) mx = sh;
       if (counts) counts[(size_t)b * K + k] = cnt[k] + ((g_mutation == 9 && k == 0) ? 1 : 0);
     }
+    free(sum);
+    free(cnt);
   }
-  free(sum);
-  free(cnt);
   if (maxshift) *maxshift = mx;
-  return 0;
+  return rc;
 }
 
 /* sum over b,i of ||x[b,i] - c[b,id]||^2 (squared error objective). */

@@ -1,0 +1,89 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol that
+include/fk.h declares, and rejects bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "fk.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fk_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = _declared()
+    for n in ["fk_assign", "fk_update", "fk_lloyd", "fk_sort", "fk_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import clustering_flashassign_b200 as fk
+    for name in _declared():
+        assert hasattr(fk.lib, name), f"libfk.so does not export {name}"
+    assert sorted(fk.EXPORTS) == _declared()
+
+
+def test_status_strings_and_version():
+    import clustering_flashassign_b200 as fk
+    assert fk.fk_status_string(fk.FK_OK) == "ok"
+    assert fk.fk_status_string(fk.FK_EINVAL) == "invalid argument"
+    assert fk.fk_status_string(fk.FK_ETIMEOUT) == "kernel wait timed out"
+    assert fk.fk_status_string(99) == "unknown status"
+    assert fk.fk_version() >= 100
+
+
+@pytest.mark.parametrize("B,N,K,d,dtype,why", [
+    (0, 10, 2, 8, 1, "positive"),
+    (1, 0, 2, 8, 1, "positive"),
+    (1, 10, 0, 8, 1, "positive"),
+    (1, 10, 11, 8, 1, "K must not exceed N"),
+    (1, 10, 2, 12, 1, "multiple of 16 bytes"),
+    (1, 10, 2, 8, 7, "unknown dtype"),
+    (1, 1 << 31, 2, 8, 1, "below 2^31"),
+])
+def test_argument_validation_happens_on_the_host(B, N, K, d, dtype, why):
+    import clustering_flashassign_b200 as fk
+    L = fk.lib
+    dummy = ctypes.c_void_p(0x1000)
+    st = L.fk_assign(dummy, dummy, B, N, K, d, dtype, dummy, None)
+    assert st == fk.FK_EINVAL
+    assert why in fk.fk_last_error()
+    st = L.fk_update(dummy, dummy, B, N, K, d, dummy, None, None, dtype, None)
+    assert st == fk.FK_EINVAL
+
+
+def test_null_and_misaligned_pointers_are_rejected():
+    import clustering_flashassign_b200 as fk
+    L = fk.lib
+    st = L.fk_assign(None, ctypes.c_void_p(0x1000), 1, 10, 2, 8, 1, ctypes.c_void_p(0x1000), None)
+    assert st == fk.FK_EINVAL and "x is NULL" in fk.fk_last_error()
+    st = L.fk_assign(ctypes.c_void_p(0x1008), ctypes.c_void_p(0x1000), 1, 10, 2, 8, 1,
+                     ctypes.c_void_p(0x1000), None)
+    assert st == fk.FK_EINVAL and "16-byte aligned" in fk.fk_last_error()
+    shape = fk.FkShape(1, 10, 2, 8, 1)
+    st = L.fk_lloyd(ctypes.byref(shape), ctypes.c_void_p(0x1000), None, 3, 0.0,
+                    ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1000), None, None, None)
+    assert st == fk.FK_EINVAL and "init_centers" in fk.fk_last_error()
+    st = L.fk_lloyd(None, None, None, 3, 0.0, None, None, None, None, None)
+    assert st == fk.FK_EINVAL
+
+
+def test_unsupported_shapes():
+    import clustering_flashassign_b200 as fk
+    L = fk.lib
+    d = ctypes.c_void_p(0x1000)
+    assert L.fk_assign(d, d, 70000, 10, 2, 8, 1, d, None) == fk.FK_EUNSUPPORTED
+    assert L.fk_sort(d, 1, 1 << 26, (1 << 24) + 1, None, None, d, None) == fk.FK_EUNSUPPORTED
+
+
+def test_binding_rejects_noncontiguous_tensors():
+    import torch
+    import clustering_flashassign_b200 as fk
+    x = torch.zeros(2, 16, 8, dtype=torch.float16).transpose(0, 1)
+    with pytest.raises(ValueError):
+        fk.fk_assign(x, torch.zeros(16, 2, 8, dtype=torch.float16), torch.zeros(16, 2, dtype=torch.int32))
