@@ -1,0 +1,400 @@
+"""Benchmark: exact batched Lloyd's K-Means on B200 through libfk.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fk|reference]
+
+Workload (the API shape of the flash-kmeans functional example): B=32
+independent problems, N=75600 points, d=128, K=1000 centroids, fp16 points
+~ N(0, 1) i.i.d., initial centroids = a seeded index set of points, up to 20
+Lloyd iterations with tol = 1e-4 on the max centroid shift.
+
+One step = one fk_lloyd call (the whole hot path: FlashAssign, counting sort,
+segment reduce, finalize, tol check) on device-resident points.  value = Lloyd
+iterations per second over all ranks (each rank runs its own B=32 problem:
+weak scaling, no data-path collective).  The points (619 MB) exceed the 126 MB
+L2, so no flush is needed between steps.
+
+Also reported: the FlashAssign kernel's achieved TFLOP/s against the measured
+tensor peak (CUDA events around every launch, on the launching stream), the
+update's GB/s against measured HBM bandwidth, the end-to-end rate through the
+C ABI with pinned host buffers (host->device copy of the points and
+device->host copy of ids and centroids inside every step), SM clocks sampled
+during the timed region, and the fp64 CPU checker timed on a bounded sample.
+
+--impl reference times that checker as the reference arm (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "api"
+METRIC = "Lloyd iter/s at B32·N75600·K1000·d128 fp16; assign TFLOP/s; update GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ["fk_assign_tc.cu", "fk_sm100.cuh", "fk_internal.h"]:
+        with open(os.path.join(ROOT, "clustering_flashassign_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per FlashAssign launch from the committed ncu summary, if it
+    was taken on the current kernel source (its hash is recorded there)."""
+    p = os.path.join(ROOT, "profiles", "flash_assign_api.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m_hash = re.search(r"kernel source hash:\s*([0-9a-f]{16})", txt)
+    m_bytes = re.search(r"dram bytes per full launch:\s*([0-9.eE+]+)", txt)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [r for r in rows if r[0] > 0.5 * r[1]] or rows
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[2][5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def make_inputs(rank):
+    import synthdata
+    w = synthdata.WORKLOADS[WORKLOAD]
+    w = synthdata.scaled(w, seed=w.seed + 7919 * rank, init_seed=w.init_seed + 100 * rank)
+    x, idx, init = synthdata.make(w)
+    return w, x, init
+
+
+def cpu_oracle_sample(x, init, w, batches, threads=0):
+    """One Lloyd iteration of the fp64 checker on `batches` of the workload."""
+    import oracle
+    import synthdata
+    xs = x[:batches].copy()
+    c = synthdata.to_f64(init[:batches], w.dtype)
+    t0 = time.perf_counter()
+    chat = oracle.round_to(c, w.dtype)
+    ids, _, _ = oracle.assign(xs, w.dtype, chat, nthreads=threads)
+    oracle.update(xs, w.dtype, ids, c)
+    return time.perf_counter() - t0
+
+
+def run_reference(args, rank):
+    """Reference arm: the fp64 CPU checker on a bounded sample (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    w, x, init = make_inputs(0)
+    batches = 1
+    for _ in range(args.warmup):
+        cpu_oracle_sample(x, init, w, batches)
+    times = [cpu_oracle_sample(x, init, w, batches) for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    value = 1.0 / (t * w.B / batches)
+    cores = oracle.max_threads()
+    sample = (f"one Lloyd iteration (assign + update) of {batches} of the {w.B} batches per step, "
+              f"extrapolated linearly to all {w.B}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "iter/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{WORKLOAD}: B={w.B} N={w.N} K={w.K} d={w.d} {w.dtype}",
+                       "parallelism": "host threads"},
+            "cpu_baseline": {"value": value, "unit": "iter/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "iter/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_fk(args, rank, world, local_rank, dist):
+    import numpy as np
+    import torch
+
+    import clustering_flashassign_b200 as fk
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w, x, init = make_inputs(rank)
+    xd = torch.from_numpy(x).to(dev)
+    initd = torch.from_numpy(init).to(dev)
+    ids = torch.empty((w.B, w.N), dtype=torch.int32, device=dev)
+    centers = torch.empty((w.B, w.K, w.d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return fk.fk_lloyd(xd, initd, w.iters, w.tol, ids, centers)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+
+    fk.fk_profile_read(reset=True)
+    fk.fk_profile_enable(True)
+    launches0 = fk.fk_launch_count()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    iters_total = 0
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        start.record(stream)
+        for _ in range(args.steps):
+            iters_total += step()
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+    fk.fk_profile_enable(False)
+    prof = fk.fk_profile_read(reset=True)
+    launches = fk.fk_launch_count() - launches0
+    ms = start.elapsed_time(stop)
+    clocks = clk.summary()
+
+    if dist is not None:
+        t = torch.tensor([ms, float(iters_total)], device=dev, dtype=torch.float64)
+        tmax = t.clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        tsum = t.clone()
+        dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
+        ms_max = float(tmax[0])
+        iters_all = float(tsum[1])
+    else:
+        ms_max, iters_all = ms, float(iters_total)
+
+    # end to end through the C ABI with pinned host buffers
+    xh = torch.from_numpy(x).pin_memory()
+    inith = torch.from_numpy(init).pin_memory()
+    idsh = torch.empty((w.B, w.N), dtype=torch.int32).pin_memory()
+    cenh = torch.empty((w.B, w.K, w.d), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        return fk.fk_lloyd(xh, inith, w.iters, w.tol, idsh, cenh, host_mode=fk.FK_HOST_RESIDENT)
+
+    e2e_step()
+    e_steps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_iters = 0
+    e0.record(stream)
+    for _ in range(e_steps):
+        e_iters += e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e_ms, float(e_iters)], device=dev, dtype=torch.float64)
+        tmax = t.clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        tsum = t.clone()
+        dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
+        e_ms, e_iters = float(tmax[0]), float(tsum[1])
+    h2d = x.nbytes + init.nbytes
+    d2h = w.B * w.N * 4 + w.B * w.K * w.d * 4
+
+    if rank != 0:
+        return
+
+    peaks, src = load_peaks()
+    flop = 2.0 * w.B * w.N * w.K * w.d
+    a_ms = prof["assign_ms"] / max(1, prof["assign_launches"])
+    achieved = flop / (a_ms * 1e-3) / 1e12
+    peak_t = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])  # fp16 rate = bf16 rate
+    traffic = recorded_traffic()
+    s = 2 if w.dtype != "f32" else 4
+    upd_bytes = (w.B * w.N * w.d * s + 8 * w.B * w.N + 8 * w.B * w.N + 16 * w.B * w.K * w.d
+                 + 2 * w.B * w.K * w.d + 12 * w.B * w.K)
+    upd_ms = (prof["sort_ms"] + prof["reduce_ms"] + prof["finalize_ms"]) / max(1, prof["update_calls"])
+    upd_gbs = upd_bytes / (upd_ms * 1e-3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+
+    import oracle
+    batches = 4
+    cpu_t = cpu_oracle_sample(x, init, w, batches)
+    cpu_value = 1.0 / (cpu_t * w.B / batches)
+
+    line = {
+        "metric": METRIC,
+        "value": iters_all / (ms_max * 1e-3),
+        "unit": "iter/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD}: B={w.B} N={w.N} K={w.K} d={w.d} {w.dtype} points ~ N(0,1), "
+                               f"{w.iters} iterations max, tol={w.tol}",
+                   "B": w.B, "N": w.N, "K": w.K, "d": w.d, "iterations_per_rank": iters_total,
+                   "l2": "inputs larger than L2 (points 619 MB per rank)",
+                   "parallelism": f"independent problems, {world} rank(s)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": achieved / peak_t, "traffic": traffic,
+                     "kernel": "FlashAssign (k_flash_assign)", "ms_per_launch": a_ms,
+                     "peak_source": f"{src} bf16 dense, sustained (fp16 runs at the bf16 rate)"},
+        "kernels": {"assign_tflops": achieved, "assign_frac": achieved / peak_t,
+                    "update_gbs": upd_gbs, "update_frac_of_hbm": upd_gbs / hbm,
+                    "update_ms": upd_ms, "sort_ms": prof["sort_ms"] / max(1, prof["update_calls"]),
+                    "reduce_ms": prof["reduce_ms"] / max(1, prof["update_calls"]),
+                    "finalize_ms": prof["finalize_ms"] / max(1, prof["update_calls"]),
+                    "hbm_peak_gbs": hbm},
+        "cpu_baseline": {"value": cpu_value, "unit": "iter/s", "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": f"one Lloyd iteration of {batches} of {w.B} batches, extrapolated"},
+        "e2e": {"value": e_iters / (e_ms * 1e-3), "unit": "iter/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_kernel_case(args):
+    """Launch only one step kind on the bench workload (for profiler captures):
+    assign = fk_assign, update = fk_update, each warmup + steps times."""
+    import torch
+
+    import clustering_flashassign_b200 as fk
+    import synthdata
+    w, x, init = make_inputs(0)
+    if args.points:
+        w = synthdata.scaled(w, N=args.points)
+        x = x[:, : args.points].copy()
+    xd = torch.from_numpy(x).cuda()
+    cd = torch.from_numpy(init).cuda()
+    ids = torch.empty((w.B, w.N), dtype=torch.int32, device="cuda")
+    fk.fk_assign(xd, cd, ids)
+    centers = cd.float()
+    counts = torch.empty((w.B, w.K), dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    for _ in range(args.warmup + args.steps):
+        if args.kernel_case == "assign":
+            fk.fk_assign(xd, cd, ids)
+        else:
+            fk.fk_update(xd, ids, centers, counts)
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel_case": args.kernel_case, "B": w.B, "N": w.N, "K": w.K, "d": w.d,
+                      "launches": fk.fk_launch_count(), "device_error": fk.fk_device_error()}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="fk", choices=["fk", "reference"])
+    ap.add_argument("--kernel-case", default=None, choices=["assign", "update"],
+                    help="launch only this step (profiler captures); prints no bench line")
+    ap.add_argument("--points", type=int, default=0, help="with --kernel-case: points per batch")
+    args = ap.parse_args()
+    world = env_int("WORLD_SIZE", 1)
+    rank = env_int("RANK", 0)
+    local_rank = env_int("LOCAL_RANK", 0)
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if args.kernel_case:
+        run_kernel_case(args)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    try:
+        run_fk(args, rank, world, local_rank, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
