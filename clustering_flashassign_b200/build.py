@@ -1,6 +1,6 @@
 """Build libfk.so (the CUDA library behind include/fk.h) in-tree for sm_100a.
 
-    python -m clustering_flashassign_b200.build [--force] [--verbose]
+    python clustering_flashassign_b200/build.py [--force] [--verbose]
 
 Each csrc/*.cu is compiled to an object with nvcc (-gencode
 arch=compute_100a,code=sm_100a -lineinfo -O3), then linked into a shared
