@@ -27,8 +27,8 @@ FK_HOST_AUTO, FK_HOST_RESIDENT, FK_HOST_STREAM = 0, 1, 2
 
 DTYPES = {torch.float32: FK_F32, torch.float16: FK_F16, torch.bfloat16: FK_BF16}
 
-EXPORTS = ["fk_assign", "fk_update", "fk_sort", "fk_lloyd", "fk_status_string", "fk_last_error",
-           "fk_device_error", "fk_release", "fk_profile_enable", "fk_profile_read",
+EXPORTS = ["fk_assign", "fk_update", "fk_sort", "fk_lloyd", "fk_assign_noalloc", "fk_status_string",
+           "fk_last_error", "fk_device_error", "fk_release", "fk_profile_enable", "fk_profile_read",
            "fk_launch_count", "fk_version"]
 
 
@@ -57,13 +57,14 @@ class FkProfile(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libfk.so not built at {LIB_PATH}; run python -m clustering_flashassign_b200.build")
+        raise ImportError(f"libfk.so not built at {LIB_PATH}; run python clustering_flashassign_b200/build.py")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, LL, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
     sig = {
         "fk_assign": (I, [P, P, I, LL, I, I, I, P, P]),
         "fk_update": (I, [P, P, I, LL, I, I, P, P, P, I, P]),
         "fk_sort": (I, [P, I, LL, I, P, P, P, P]),
+        "fk_assign_noalloc": (I, [P, P, I, LL, I, I, I, P, P]),
         "fk_lloyd": (I, [ctypes.POINTER(FkShape), P, P, I, F, P, P, P, ctypes.POINTER(I),
                          ctypes.POINTER(FkOptions)]),
         "fk_status_string": (ctypes.c_char_p, [I]),
@@ -119,6 +120,15 @@ def fk_assign(x: torch.Tensor, c: torch.Tensor, ids: torch.Tensor, stream=None) 
     K = c.shape[1]
     _check(lib.fk_assign(_ptr(x), _ptr(c), B, N, K, d, _dtype_code(x), _ptr(ids), _stream(stream)),
            "fk_assign")
+    return ids
+
+
+def fk_assign_noalloc(x: torch.Tensor, c: torch.Tensor, ids: torch.Tensor, stream=None) -> torch.Tensor:
+    """fk_assign that allocates no device memory (static scratch; see include/fk.h)."""
+    B, N, d = x.shape
+    K = c.shape[1]
+    _check(lib.fk_assign_noalloc(_ptr(x), _ptr(c), B, N, K, d, _dtype_code(x), _ptr(ids),
+                                 _stream(stream)), "fk_assign_noalloc")
     return ids
 
 

@@ -1,0 +1,80 @@
+// fk_assign_noalloc: FlashAssign for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc at the point where they need an
+// assignment: code running under a custom or pooled allocator that owns all
+// device memory, real-time loops that forbid allocation (and the implicit
+// device synchronization that cudaFree can bring), or hosts that only hand
+// out pre-registered buffers.  fk_assign keeps its scratch (the ||c||^2
+// vector and the kernel error word) in a per-stream workspace that it grows
+// with cudaMalloc; this variant instead uses one file-scope static device
+// array, so a call allocates nothing.  The caller still passes the inputs and
+// the output.
+//
+// The array lives on every GPU that loads the library until the process
+// exits.  Its size caps B * Kpad (Kpad = K rounded up to 256) at
+// kNoAllocMaxCn floats.  Host code cannot use the array's name as a device
+// address; the address is looked up once per device with
+// cudaGetSymbolAddress while that device is current.
+#include <mutex>
+
+#include "fk_internal.h"
+
+namespace fk {
+namespace {
+
+constexpr long long kNoAllocMaxCn = 1LL << 20;  // floats of ||c||^2 (4 MiB)
+constexpr int kNoAllocHeader = 64;              // floats reserved for the error word
+
+// [0, kNoAllocHeader): error word (int) and padding; then B * Kpad floats of cn.
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocHeader + kNoAllocMaxCn];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_na_mu;
+float *g_na_addr[kMaxDevices] = {nullptr};
+
+int noalloc_base(float **out) {
+  int dev = 0;
+  FK_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return set_error(FK_EUNSUPPORTED, "device index above 63");
+  std::lock_guard<std::mutex> lk(g_na_mu);
+  if (!g_na_addr[dev]) {
+    void *p = nullptr;
+    FK_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    g_na_addr[dev] = static_cast<float *>(p);
+  }
+  *out = g_na_addr[dev];
+  return FK_OK;
+}
+
+}  // namespace
+}  // namespace fk
+
+using namespace fk;
+
+extern "C" int fk_assign_noalloc(const void *x, const void *c, int B, long long N, int K, int d,
+                                 int dtype, int32_t *ids, fk_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype != FK_F32 && dtype != FK_F16 && dtype != FK_BF16)
+    return set_error(FK_EINVAL, "unknown dtype " + std::to_string(dtype));
+  if (B <= 0 || N <= 0 || K <= 0 || d <= 0) return set_error(FK_EINVAL, "B, N, K and d must be positive");
+  if (N > 0x7fffffffLL) return set_error(FK_EINVAL, "N must be below 2^31");
+  if ((long long)K > N) return set_error(FK_EINVAL, "K must not exceed N");
+  if (B > 65535) return set_error(FK_EUNSUPPORTED, "B above 65535");
+  if (dtype != FK_F32 && (d * 2) % 16 != 0)
+    return set_error(FK_EINVAL, "fp16/bf16 rows must be a multiple of 16 bytes (d % 8 == 0)");
+  if (!x || !c || !ids) return set_error(FK_EINVAL, "x, c and ids must not be NULL");
+  const bool tc = dtype != FK_F32;
+  if (tc && ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(c)) & 15u))
+    return set_error(FK_EINVAL, "x and c must be 16-byte aligned");
+  if (!tc) return launch_assign_f32((const float *)x, (const float *)c, B, N, K, d, ids, s);
+  const long long Kpad = kpad_of(K);
+  if ((long long)B * Kpad > kNoAllocMaxCn)
+    return set_error(FK_EUNSUPPORTED, "fk_assign_noalloc: B * ceil(K/256)*256 exceeds 1048576");
+  float *base = nullptr;
+  FK_TRY(noalloc_base(&base));
+  int *err = reinterpret_cast<int *>(base);
+  float *cn = base + kNoAllocHeader;
+  FK_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));  // start each call with a clear error word
+  FK_TRY(launch_prep_cn(c, dtype, B, K, d, Kpad, cn, s));
+  return launch_assign_tc(x, c, cn, dtype, B, N, K, d, Kpad, ids, err, s);
+}

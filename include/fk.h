@@ -165,6 +165,30 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
              float tol, int32_t *ids, float *centers, fk_stream_t stream, int *iters_run,
              const fk_options *opts);
 
+/*
+ * fk_assign_noalloc -- fk_assign for callers that cannot allocate device
+ * memory (no counterpart in the paper; it is an interface addition).
+ * Same arguments, layouts and result as fk_assign.  Callers that run under an
+ * allocator owning all device memory, or in loops where allocation (and the
+ * synchronization a cudaFree can bring) is not allowed, cannot let fk_assign
+ * grow its workspace; this call allocates nothing.  Its scratch (the
+ * ||c||^2 vector and the kernel error word) is one static device array of
+ * 4 MiB + 256 bytes that every GPU loading the library holds until the
+ * process exits.
+ *   Limit: B * Kpad <= 1048576 for fp16 / bf16, Kpad = K rounded up to a
+ *   multiple of 256; larger shapes return FK_EUNSUPPORTED.  fp32 needs no
+ *   scratch and has no such limit.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   All calls on a device share the array: calls that overlap on the GPU
+ *   (e.g. on two streams) race and may return wrong ids.  The error word is
+ *   cleared at the start of each call; a bounded-wait timeout inside this
+ *   variant is recorded there and is not reported by fk_device_error().
+ */
+int fk_assign_noalloc(const void *x, const void *c, int B, long long N, int K, int d, int dtype,
+                      int32_t *ids, fk_stream_t stream);
+
 /* Static text for a status code. */
 const char *fk_status_string(int status);
 

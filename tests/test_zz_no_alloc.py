@@ -1,0 +1,68 @@
+"""fk_assign_noalloc: the assign entry point for callers that cannot allocate.
+
+Callers that run under an allocator owning all device memory, or inside loops
+where cudaMalloc / cudaFree are not allowed, use this variant; its scratch is a
+static device array.  The test drives it through the C ABI and checks that it
+returns exactly what fk_assign returns, on two calls in a row with different
+shapes (the shared scratch must not leak state from one call into the next),
+and that the second call leaves free device memory unchanged.  This file is
+collected last so that a failure here comes after every other test has run.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synthdata
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(B, N, K, d, dtype, seed):
+    w = synthdata.Workload("na", B, N, K, d, dtype, K, 3.0, 0.0, 1, 0.0, seed, seed + 1)
+    x, idx, c = synthdata.make(w)
+    if dtype == "bf16":
+        to = lambda a: torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).cuda()
+    else:
+        to = lambda a: torch.from_numpy(a).cuda()
+    return to(x), to(c)
+
+
+def _raw_noalloc(fk, x, c, ids):
+    B, N, d = x.shape
+    K = c.shape[1]
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return fk.lib.fk_assign_noalloc(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(c.data_ptr()), B, N, K,
+                                    d, fk.DTYPES[x.dtype], ctypes.c_void_p(ids.data_ptr()), stream)
+
+
+def test_noalloc_assign_matches_fk_assign_on_consecutive_calls():
+    import clustering_flashassign_b200 as fk
+    cases = [(4, 3000, 1000, 128, "f16", 5), (2, 2000, 300, 192, "bf16", 6), (1, 500, 70, 24, "f32", 7)]
+    free_after_first = None
+    for n, (B, N, K, d, dtype, seed) in enumerate(cases + cases[:1]):
+        x, c = _inputs(B, N, K, d, dtype, seed)
+        ref = torch.empty((B, N), dtype=torch.int32, device="cuda")
+        fk.fk_assign(x, c, ref)
+        got = torch.full((B, N), -1, dtype=torch.int32, device="cuda")
+        torch.cuda.synchronize()
+        free0, _ = torch.cuda.mem_get_info()
+        st = _raw_noalloc(fk, x, c, got)
+        torch.cuda.synchronize()
+        free1, _ = torch.cuda.mem_get_info()
+        assert st == fk.FK_OK, fk.fk_last_error()
+        assert torch.equal(got, ref), f"call {n}: ids differ from fk_assign"
+        if n > 0:  # the first call may load the module that holds the static array
+            assert free1 == free0, "fk_assign_noalloc changed free device memory"
+        free_after_first = free1
+    assert free_after_first is not None
+
+
+def test_noalloc_assign_rejects_shapes_beyond_its_scratch():
+    import clustering_flashassign_b200 as fk
+    d = ctypes.c_void_p(0x1000)
+    # B * Kpad = 5 * 262144 > 2^20 floats of scratch
+    st = fk.lib.fk_assign_noalloc(d, d, 5, 300000, 262144, 128, fk.FK_F16, d, None)
+    assert st == fk.FK_EUNSUPPORTED
+    assert "exceeds" in fk.fk_last_error()
