@@ -52,19 +52,16 @@ int read_device_error(Workspace *ws, cudaStream_t s) {
   return set_error(FK_EINVAL, "an id outside [0, K) reached the update");
 }
 
-// Sorted keys + perm for `sort_entries` positions and fp32 sums for
-// `sum_rows` centroids of d; the sums stay all-zero between calls (the
-// finalize clears what it reads; a fresh or dirty buffer is cleared here).
-int prepare_update(Workspace *ws, long long sort_entries, long long sum_rows, int d, cudaStream_t s) {
-  FK_TRY(ensure(ws->keys_a, (size_t)sort_entries * sizeof(int32_t)));
-  FK_TRY(ensure(ws->vals_a, (size_t)sort_entries * sizeof(int32_t)));
-  void *old = ws->sums.p;
-  FK_TRY(ensure(ws->sums, (size_t)sum_rows * d * sizeof(float)));
-  if (ws->sums.p != old) ws->sums_dirty = true;
-  if (ws->sums_dirty) {
-    FK_CUDA(cudaMemsetAsync(ws->sums.p, 0, ws->sums.bytes, s));
-    ws->sums_dirty = false;
-  }
+// Scratch of one update over B batches of n sorted positions: sorted keys,
+// perm, segment offsets, owner partial sums (B, K, d) and continuation
+// partials (B, pieces, d).  Nothing here needs clearing: every value read is
+// written by the same update first.
+int prepare_update(Workspace *ws, int B, long long n, int K, int d) {
+  FK_TRY(ensure(ws->keys_a, (size_t)B * n * sizeof(int32_t)));
+  FK_TRY(ensure(ws->vals_a, (size_t)B * n * sizeof(int32_t)));
+  FK_TRY(ensure(ws->offsets, (size_t)B * K * sizeof(int32_t)));
+  FK_TRY(ensure(ws->sums, (size_t)B * K * d * sizeof(float)));
+  FK_TRY(ensure(ws->first, (size_t)B * pieces_of(n) * d * sizeof(float)));
   return FK_OK;
 }
 
@@ -79,29 +76,22 @@ int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long
     FK_TRY(ensure(ws->counts, (size_t)B * K * sizeof(int32_t)));
     counts = (int32_t *)ws->counts.p;
   }
-  FK_TRY(prepare_update(ws, (long long)B * N, (long long)B * K, d, s));
+  FK_TRY(prepare_update(ws, B, N, K, d));
   FK_CUDA(cudaMemsetAsync(ws->maxshift, 0, sizeof(unsigned), s));
   int32_t *keys = (int32_t *)ws->keys_a.p, *perm = (int32_t *)ws->vals_a.p;
+  int32_t *offsets = (int32_t *)ws->offsets.p;
+  float *sums = (float *)ws->sums.p, *first = (float *)ws->first.p;
   {
     PhaseTimer t(PH_SORT, s);
-    FK_TRY(run_sort(ws, ids, B, N, K, counts, nullptr, perm, keys, false, s));
+    FK_TRY(run_sort(ws, ids, B, N, K, counts, offsets, perm, keys, s));
   }
-  int st;
   {
     PhaseTimer t(PH_REDUCE, s);
-    st = launch_segreduce(x, dtype, keys, perm, B, N, K, d, (float *)ws->sums.p, s);
+    FK_TRY(launch_segreduce(x, dtype, keys, perm, B, N, K, d, sums, first, s));
   }
-  if (st != FK_OK) {
-    ws->sums_dirty = true;
-    return st;
-  }
-  {
-    PhaseTimer t(PH_FINALIZE, s);
-    st = launch_finalize((float *)ws->sums.p, counts, centers, ch, cn, dtype, B, K, d, Kpad,
-                         ws->maxshift, s);
-  }
-  if (st != FK_OK) ws->sums_dirty = true;
-  return st;
+  PhaseTimer t(PH_FINALIZE, s);
+  return launch_finalize(sums, first, pieces_of(N), counts, offsets, centers, ch, cn, dtype, B, K,
+                         d, Kpad, ws->maxshift, true, s);
 }
 
 int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const float *cn, int B,
@@ -156,17 +146,24 @@ int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void
     ch = ws->ch.p;
     cn = (float *)ws->cn.p;
   }
-  FK_TRY(ensure(ws->counts, (size_t)B * K * sizeof(int32_t)));
-  int32_t *counts = (int32_t *)ws->counts.p;
+  // per chunk: counts, offsets, owner / continuation partials (one batch);
+  // per iteration: running sums and counts of every batch
+  FK_TRY(ensure(ws->counts, (size_t)K * sizeof(int32_t)));
+  FK_TRY(ensure(ws->gsum, (size_t)B * K * d * sizeof(float)));
+  FK_TRY(ensure(ws->gcounts, (size_t)B * K * sizeof(int32_t)));
+  int32_t *counts = (int32_t *)ws->counts.p, *gcounts = (int32_t *)ws->gcounts.p;
+  float *gsum = (float *)ws->gsum.p;
   FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cn, s));
-  FK_TRY(prepare_update(ws, chunk, (long long)B * K, d, s));
-  float *sums = (float *)ws->sums.p;
+  FK_TRY(prepare_update(ws, 1, chunk, K, d));
+  float *sums = (float *)ws->sums.p, *first = (float *)ws->first.p;
   int32_t *keys = (int32_t *)ws->keys_a.p, *perm = (int32_t *)ws->vals_a.p;
+  int32_t *offsets = (int32_t *)ws->offsets.p;
   long long job = 0;
   int it = 0;
   for (it = 0; it < max_iter; ++it) {
     note_update_call();
-    FK_CUDA(cudaMemsetAsync(counts, 0, (size_t)B * K * sizeof(int32_t), s));
+    FK_CUDA(cudaMemsetAsync(gcounts, 0, (size_t)B * K * sizeof(int32_t), s));
+    FK_CUDA(cudaMemsetAsync(gsum, 0, (size_t)B * K * d * sizeof(float), s));
     FK_CUDA(cudaMemsetAsync(ws->maxshift, 0, sizeof(unsigned), s));
     for (int b = 0; b < B; ++b) {
       for (long long ci = 0; ci < per_b; ++ci, ++job) {
@@ -186,26 +183,21 @@ int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void
                                   Kpad, idc, s));
         {
           PhaseTimer t(PH_SORT, s);
-          FK_TRY(run_sort(ws, idc, 1, nc, K, counts + (size_t)b * K, nullptr, perm, keys, true, s));
+          FK_TRY(run_sort(ws, idc, 1, nc, K, counts, offsets, perm, keys, s));
         }
         {
           PhaseTimer t(PH_REDUCE, s);
-          int st = launch_segreduce(xb, dtype, keys, perm, 1, nc, K, d, sums + (size_t)b * K * d, s);
-          if (st != FK_OK) {
-            ws->sums_dirty = true;
-            return st;
-          }
+          FK_TRY(launch_segreduce(xb, dtype, keys, perm, 1, nc, K, d, sums, first, s));
+          FK_TRY(launch_accumulate(sums, first, pieces_of(nc), counts, offsets, K, d,
+                                   gsum + (size_t)b * K * d, gcounts + (size_t)b * K, s));
         }
         FK_CUDA(cudaEventRecord(ws->freed[buf], s));
       }
     }
     {
       PhaseTimer t(PH_FINALIZE, s);
-      int st = launch_finalize(sums, counts, cen_dev, ch, cn, dtype, B, K, d, Kpad, ws->maxshift, s);
-      if (st != FK_OK) {
-        ws->sums_dirty = true;
-        return st;
-      }
+      FK_TRY(launch_finalize(gsum, nullptr, 0, gcounts, nullptr, cen_dev, ch, cn, dtype, B, K, d,
+                             Kpad, ws->maxshift, false, s));
     }
     if (tol > 0.f || verbose) {
       float ms = 0.f;
@@ -272,7 +264,7 @@ int fk_sort(const int32_t *ids, int B, long long N, int K, int32_t *counts, int3
   Workspace *ws;
   FK_TRY(workspace_for(s, &ws));
   PhaseTimer t(PH_SORT, s);
-  return run_sort(ws, ids, B, N, K, counts, offsets, perm, nullptr, false, s);
+  return run_sort(ws, ids, B, N, K, counts, offsets, perm, nullptr, s);
 }
 
 int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int max_iter,

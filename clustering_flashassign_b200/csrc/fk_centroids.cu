@@ -1,5 +1,6 @@
-// Centroid-side kernels: ||c||^2 preparation, fk_lloyd initialisation and the
-// update's finalize step (mean, empty-cluster rule, shift, dtype copy).
+// Centroid-side kernels: ||c||^2 preparation, fk_lloyd initialisation, the
+// update's finalize step (mean, empty-cluster rule, shift, dtype copy) and the
+// per-chunk accumulation of the streamed path.
 //
 // Update rule: each centroid becomes the mean of the points assigned to it
 // ("Flash-KMeans: IO感知的精确K-Means", section "什么是 Flash-KMeans"); a
@@ -7,6 +8,12 @@
 // the tol test of the functional API ("flash-kmeans and the return of exact
 // K-Means on the GPU", section "Exact K-Means, with the assignment step
 // written in Triton") is the L2 norm of new - old, maximised over b, k.
+//
+// Layout of the work: one warp per centroid; lane l handles elements
+// 4l..4l+3, 4l+128.. (d % 4 == 0) or l, l+32, ... otherwise.  ||c||^2 is
+// accumulated in that element order and then butterfly-reduced across lanes,
+// identically in every kernel here, so the value the Lloyd loop fuses into its
+// finalize equals the one fk_assign computes from the same dtype centroids.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -32,91 +39,151 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 constexpr int kWarpsPerBlock = 8;
+constexpr float kInf = __builtin_huge_valf();
 
-// One warp per centroid.  cn from the stored (already rounded) values.
-template <typename T>
+// Element loop shared by every kernel: f(j, n) handles elements j .. j+n-1.
+template <bool V4, typename F>
+__device__ __forceinline__ void for_lane_elems(int d, int lane, F &&f) {
+  if (V4) {
+    for (int j = lane * 4; j < d; j += 128) f(j, 4);
+  } else {
+    for (int j = lane; j < d; j += 32) f(j, 1);
+  }
+}
+
+template <typename T, bool V4>
 __global__ void k_prep_cn(const T *__restrict__ c, int B, int K, int d, long long Kpad,
                           float *__restrict__ cn) {
-  long long w = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  int lane = threadIdx.x & 31;
-  long long total = (long long)B * Kpad;
-  if (w >= total) return;
-  int b = (int)(w / Kpad);
-  int k = (int)(w % Kpad);
+  const long long w = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)B * Kpad) return;
+  const int b = (int)(w / Kpad), k = (int)(w % Kpad);
   if (k >= K) {
-    if (lane == 0) cn[w] = __int_as_float(0x7f800000);  // +inf: padded columns never win
+    if (lane == 0) cn[w] = kInf;  // padded columns never win
     return;
   }
   const T *row = c + ((size_t)b * K + k) * d;
   float s = 0.f;
-  for (int j = lane; j < d; j += 32) {
-    float v = to_f<T>(row[j]);
-    s = fmaf(v, v, s);
-  }
+  for_lane_elems<V4>(d, lane, [&](int j, int n) {
+    for (int e = 0; e < n; ++e) {
+      const float v = to_f<T>(row[j + e]);
+      s = fmaf(v, v, s);
+    }
+  });
   s = warp_sum(s);
   if (lane == 0) cn[w] = s;
 }
 
-template <typename T>
+template <typename T, bool V4>
 __global__ void k_init(const T *__restrict__ init, int B, int K, int d, long long Kpad,
                        float *__restrict__ master, T *__restrict__ ch, float *__restrict__ cn) {
-  long long w = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  int lane = threadIdx.x & 31;
-  long long total = (long long)B * Kpad;
-  if (w >= total) return;
-  int b = (int)(w / Kpad);
-  int k = (int)(w % Kpad);
+  const long long w = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)B * Kpad) return;
+  const int b = (int)(w / Kpad), k = (int)(w % Kpad);
   if (k >= K) {
-    if (lane == 0 && cn) cn[w] = __int_as_float(0x7f800000);
+    if (lane == 0 && cn) cn[w] = kInf;
     return;
   }
-  size_t off = ((size_t)b * K + k) * d;
+  const size_t off = ((size_t)b * K + k) * d;
   float s = 0.f;
-  for (int j = lane; j < d; j += 32) {
-    T v = init[off + j];
-    float f = to_f<T>(v);
-    master[off + j] = f;
-    if (ch) ch[off + j] = v;
-    s = fmaf(f, f, s);
-  }
+  for_lane_elems<V4>(d, lane, [&](int j, int n) {
+    for (int e = 0; e < n; ++e) {
+      const T v = init[off + j + e];
+      const float f = to_f<T>(v);
+      master[off + j + e] = f;
+      if (ch) ch[off + j + e] = v;
+      s = fmaf(f, f, s);
+    }
+  });
   s = warp_sum(s);
   if (lane == 0 && cn) cn[w] = s;
 }
 
-// One warp per centroid: divide, keep empty clusters, shift, dtype copy, cn,
-// and clear the sums for the next accumulation.
-template <typename T>
-__global__ void k_finalize(float *__restrict__ sums, const int32_t *__restrict__ counts,
-                           float *__restrict__ centers, T *__restrict__ ch, float *__restrict__ cn,
-                           int B, int K, int d, long long Kpad, unsigned *__restrict__ maxshift) {
-  long long w = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  int lane = threadIdx.x & 31;
-  if (w >= (long long)B * K) return;
-  int b = (int)(w / K);
-  int k = (int)(w % K);
-  int cnt = counts[w];
-  size_t off = (size_t)w * d;
-  float shift2 = 0.f, nrm = 0.f;
-  for (int j = lane; j < d; j += 32) {
-    float old = centers[off + j];
-    float s = sums[off + j];
-    float nv = cnt > 0 ? s / (float)cnt : old;
-    float t = nv - old;
-    shift2 = fmaf(t, t, shift2);
-    centers[off + j] = nv;
-    sums[off + j] = 0.f;
-    if (ch) {
-      T r = from_f<T>(nv);
-      ch[off + j] = r;
-      float rf = to_f<T>(r);
-      nrm = fmaf(rf, rf, nrm);
+// Sum of cluster w: the owner piece's partial plus the continuation partials
+// of the following pieces, in piece order (see fk_reduce.cu).
+template <bool FROM_PIECES>
+__device__ __forceinline__ float seg_sum(const float *sums, const float *first, size_t w_off,
+                                         size_t first_b, int d, int p0, int pl, int j) {
+  float s = sums[w_off + j];
+  if (FROM_PIECES)
+    for (int p = p0 + 1; p <= pl; ++p) s += first[first_b + (size_t)p * d + j];
+  return s;
+}
+
+template <typename T, bool V4, bool FROM_PIECES>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+    k_finalize(const float *__restrict__ sums, const float *__restrict__ first, int pieces,
+               const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets,
+               float *__restrict__ centers, T *__restrict__ ch, float *__restrict__ cn, int B, int K,
+               int d, long long Kpad, unsigned *__restrict__ maxshift) {
+  __shared__ float wmax[kWarpsPerBlock];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float my_max = 0.f;
+  for (long long w = (long long)blockIdx.x * kWarpsPerBlock + warp; w < (long long)B * K;
+       w += (long long)gridDim.x * kWarpsPerBlock) {
+    const int b = (int)(w / K), k = (int)(w % K);
+    const int cnt = counts[w];
+    int p0 = 0, pl = -1;
+    if (FROM_PIECES && cnt > 0) {
+      const int off = offsets[w];
+      p0 = off / kPiece;
+      pl = (off + cnt - 1) / kPiece;
     }
+    const size_t w_off = (size_t)w * d;
+    const size_t first_b = (size_t)b * pieces * d;
+    float shift2 = 0.f, nrm = 0.f;
+    for_lane_elems<V4>(d, lane, [&](int j, int n) {
+      for (int e = 0; e < n; ++e) {
+        const float old = centers[w_off + j + e];
+        float nv = old;
+        if (cnt > 0) nv = seg_sum<FROM_PIECES>(sums, first, w_off, first_b, d, p0, pl, j + e) / (float)cnt;
+        const float t = nv - old;
+        shift2 = fmaf(t, t, shift2);
+        centers[w_off + j + e] = nv;
+        if (ch) {
+          const T r = from_f<T>(nv);
+          ch[w_off + j + e] = r;
+          const float rf = to_f<T>(r);
+          nrm = fmaf(rf, rf, nrm);
+        }
+      }
+    });
+    shift2 = warp_sum(shift2);
+    nrm = warp_sum(nrm);
+    if (lane == 0 && cn) cn[(size_t)b * Kpad + k] = nrm;
+    my_max = fmaxf(my_max, sqrtf(shift2));
   }
-  shift2 = warp_sum(shift2);
-  nrm = warp_sum(nrm);
-  if (lane == 0) {
-    if (cn) cn[(size_t)b * Kpad + k] = nrm;
-    if (maxshift) atomicMax(maxshift, __float_as_uint(sqrtf(shift2)));
+  if (lane == 0) wmax[warp] = my_max;
+  __syncthreads();
+  if (threadIdx.x == 0 && maxshift) {
+    float m = 0.f;
+    for (int i = 0; i < kWarpsPerBlock; ++i) m = fmaxf(m, wmax[i]);
+    atomicMax(maxshift, __float_as_uint(m));  // non-negative floats order as unsigned ints
+  }
+}
+
+// Streamed path: fold one chunk's segment sums and counts into the running
+// totals of its batch (chunks are folded in order, so the totals are
+// reproducible).
+template <bool V4>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+    k_accumulate(const float *__restrict__ sums, const float *__restrict__ first, int pieces,
+                 const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets, int K,
+                 int d, float *__restrict__ gsum, int32_t *__restrict__ gcounts) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (long long k = (long long)blockIdx.x * kWarpsPerBlock + warp; k < K;
+       k += (long long)gridDim.x * kWarpsPerBlock) {
+    const int cnt = counts[k];
+    if (cnt == 0) continue;
+    const int off = offsets[k];
+    const int p0 = off / kPiece, pl = (off + cnt - 1) / kPiece;
+    const size_t w_off = (size_t)k * d;
+    for_lane_elems<V4>(d, lane, [&](int j, int n) {
+      for (int e = 0; e < n; ++e)
+        gsum[w_off + j + e] += seg_sum<true>(sums, first, w_off, 0, d, p0, pl, j + e);
+    });
+    if (lane == 0) gcounts[k] += cnt;
   }
 }
 
@@ -124,46 +191,87 @@ inline unsigned blocks_for(long long warps) {
   return (unsigned)((warps + kWarpsPerBlock - 1) / kWarpsPerBlock);
 }
 
+template <typename T>
+int prep_t(const void *c, int B, int K, int d, long long Kpad, float *cn, cudaStream_t s) {
+  const unsigned g = blocks_for((long long)B * Kpad);
+  if (d % 4 == 0) k_prep_cn<T, true><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)c, B, K, d, Kpad, cn);
+  else k_prep_cn<T, false><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)c, B, K, d, Kpad, cn);
+  count_launch();
+  FK_CUDA(cudaGetLastError());
+  return FK_OK;
+}
+
+template <typename T>
+int init_t(const void *init, int B, int K, int d, long long Kpad, float *master, void *ch,
+           float *cn, cudaStream_t s) {
+  const unsigned g = blocks_for((long long)B * Kpad);
+  if (d % 4 == 0)
+    k_init<T, true><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)init, B, K, d, Kpad, master, (T *)ch, cn);
+  else
+    k_init<T, false><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)init, B, K, d, Kpad, master, (T *)ch, cn);
+  count_launch();
+  FK_CUDA(cudaGetLastError());
+  return FK_OK;
+}
+
+template <typename T, bool FP>
+int fin_t(const float *sums, const float *first, int pieces, const int32_t *counts,
+          const int32_t *offsets, float *centers, void *ch, float *cn, int B, int K, int d,
+          long long Kpad, unsigned *maxshift, cudaStream_t s) {
+  unsigned g = blocks_for((long long)B * K);
+  const unsigned cap = (unsigned)num_sms() * 8;
+  if (g > cap) g = cap;
+  if (d % 4 == 0)
+    k_finalize<T, true, FP><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, centers,
+                                                              (T *)ch, cn, B, K, d, Kpad, maxshift);
+  else
+    k_finalize<T, false, FP><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, centers,
+                                                               (T *)ch, cn, B, K, d, Kpad, maxshift);
+  count_launch();
+  FK_CUDA(cudaGetLastError());
+  return FK_OK;
+}
+
 }  // namespace
 
 int launch_prep_cn(const void *c, int dtype, int B, int K, int d, long long Kpad, float *cn,
                    cudaStream_t s) {
-  long long warps = (long long)B * Kpad;
-  if (dtype == FK_F16)
-    k_prep_cn<__half><<<blocks_for(warps), kWarpsPerBlock * 32, 0, s>>>((const __half *)c, B, K, d, Kpad, cn);
-  else if (dtype == FK_BF16)
-    k_prep_cn<__nv_bfloat16><<<blocks_for(warps), kWarpsPerBlock * 32, 0, s>>>((const __nv_bfloat16 *)c, B, K, d, Kpad, cn);
-  else
-    k_prep_cn<float><<<blocks_for(warps), kWarpsPerBlock * 32, 0, s>>>((const float *)c, B, K, d, Kpad, cn);
-  count_launch();
-  FK_CUDA(cudaGetLastError());
-  return FK_OK;
+  if (dtype == FK_F16) return prep_t<__half>(c, B, K, d, Kpad, cn, s);
+  if (dtype == FK_BF16) return prep_t<__nv_bfloat16>(c, B, K, d, Kpad, cn, s);
+  return prep_t<float>(c, B, K, d, Kpad, cn, s);
 }
 
 int launch_init_centers(const void *init, int dtype, int B, int K, int d, long long Kpad,
                         float *master, void *ch, float *cn, cudaStream_t s) {
-  long long warps = (long long)B * Kpad;
-  if (dtype == FK_F16)
-    k_init<__half><<<blocks_for(warps), kWarpsPerBlock * 32, 0, s>>>((const __half *)init, B, K, d, Kpad, master, (__half *)ch, cn);
-  else if (dtype == FK_BF16)
-    k_init<__nv_bfloat16><<<blocks_for(warps), kWarpsPerBlock * 32, 0, s>>>((const __nv_bfloat16 *)init, B, K, d, Kpad, master, (__nv_bfloat16 *)ch, cn);
-  else
-    k_init<float><<<blocks_for(warps), kWarpsPerBlock * 32, 0, s>>>((const float *)init, B, K, d, Kpad, master, nullptr, cn);
-  count_launch();
-  FK_CUDA(cudaGetLastError());
-  return FK_OK;
+  if (dtype == FK_F16) return init_t<__half>(init, B, K, d, Kpad, master, ch, cn, s);
+  if (dtype == FK_BF16) return init_t<__nv_bfloat16>(init, B, K, d, Kpad, master, ch, cn, s);
+  return init_t<float>(init, B, K, d, Kpad, master, nullptr, cn, s);
 }
 
-int launch_finalize(float *sums, const int32_t *counts, float *centers, void *ch, float *cn,
-                    int dtype, int B, int K, int d, long long Kpad, unsigned *maxshift,
+int launch_finalize(const float *sums, const float *first, int pieces, const int32_t *counts,
+                    const int32_t *offsets, float *centers, void *ch, float *cn, int dtype, int B,
+                    int K, int d, long long Kpad, unsigned *maxshift, bool from_pieces,
                     cudaStream_t s) {
-  long long warps = (long long)B * K;
   if (dtype == FK_F16)
-    k_finalize<__half><<<blocks_for(warps), kWarpsPerBlock * 32, 0, s>>>(sums, counts, centers, (__half *)ch, cn, B, K, d, Kpad, maxshift);
-  else if (dtype == FK_BF16)
-    k_finalize<__nv_bfloat16><<<blocks_for(warps), kWarpsPerBlock * 32, 0, s>>>(sums, counts, centers, (__nv_bfloat16 *)ch, cn, B, K, d, Kpad, maxshift);
+    return from_pieces ? fin_t<__half, true>(sums, first, pieces, counts, offsets, centers, ch, cn, B, K, d, Kpad, maxshift, s)
+                       : fin_t<__half, false>(sums, first, pieces, counts, offsets, centers, ch, cn, B, K, d, Kpad, maxshift, s);
+  if (dtype == FK_BF16)
+    return from_pieces ? fin_t<__nv_bfloat16, true>(sums, first, pieces, counts, offsets, centers, ch, cn, B, K, d, Kpad, maxshift, s)
+                       : fin_t<__nv_bfloat16, false>(sums, first, pieces, counts, offsets, centers, ch, cn, B, K, d, Kpad, maxshift, s);
+  return from_pieces ? fin_t<float, true>(sums, first, pieces, counts, offsets, centers, nullptr, cn, B, K, d, Kpad, maxshift, s)
+                     : fin_t<float, false>(sums, first, pieces, counts, offsets, centers, nullptr, cn, B, K, d, Kpad, maxshift, s);
+}
+
+int launch_accumulate(const float *sums, const float *first, int pieces, const int32_t *counts,
+                      const int32_t *offsets, int K, int d, float *gsum, int32_t *gcounts,
+                      cudaStream_t s) {
+  unsigned g = blocks_for(K);
+  const unsigned cap = (unsigned)num_sms() * 8;
+  if (g > cap) g = cap;
+  if (d % 4 == 0)
+    k_accumulate<true><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, K, d, gsum, gcounts);
   else
-    k_finalize<float><<<blocks_for(warps), kWarpsPerBlock * 32, 0, s>>>(sums, counts, centers, nullptr, cn, B, K, d, Kpad, maxshift);
+    k_accumulate<false><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, K, d, gsum, gcounts);
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;

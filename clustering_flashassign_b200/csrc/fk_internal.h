@@ -25,13 +25,13 @@ constexpr int kBlockK = 64;   // elements of d per K-block (128-byte rows for 16
 inline long long kpad_of(int K) { return ((long long)K + kChunkN - 1) / kChunkN * kChunkN; }
 
 // Counting-sort geometry.
-constexpr int kSortWarps = 8;
-constexpr int kSortRounds = 16;
-constexpr int kSortTile = kSortWarps * kSortRounds * 32;  // 4096 points per CTA
+constexpr int kSortTile = 2048;    // points per sort tile (one warp walks it in order)
 constexpr int kMaxDigitBits = 12;                         // 4096 bins per pass at most
 
 // Segment-reduce geometry.
-constexpr int kPiece = 64;  // sorted positions per segment piece
+constexpr int kPiece = 128;  // sorted positions per segment piece
+
+inline int pieces_of(long long N) { return (int)((N + kPiece - 1) / kPiece); }
 
 struct DevBuf {
   void *p = nullptr;
@@ -45,9 +45,8 @@ struct Workspace {
   int *err = nullptr;             // device error word
   unsigned *maxshift = nullptr;   // device, float bits (non-negative floats order as uints)
   float *h_maxshift = nullptr;    // pinned host mirror
-  DevBuf cn, ch, sums, counts, offsets, table, keys_a, vals_a, keys_b, vals_b;
-  DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2];
-  bool sums_dirty = true;
+  DevBuf cn, ch, sums, first, counts, offsets, table, digit_off, keys_a, vals_a, keys_b, vals_b;
+  DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2], gsum, gcounts;
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
 };
@@ -96,23 +95,31 @@ int launch_prep_cn(const void *c, int dtype, int B, int K, int d, long long Kpad
 // init for fk_lloyd: master = float(init), ch = init (16-bit dtypes), cn.
 int launch_init_centers(const void *init, int dtype, int B, int K, int d, long long Kpad,
                         float *master, void *ch, float *cn, cudaStream_t s);
-// finalize: new = sums / count or old; shift max; master, ch, cn; zero sums.
-int launch_finalize(float *sums, const int32_t *counts, float *centers, void *ch, float *cn,
-                    int dtype, int B, int K, int d, long long Kpad, unsigned *maxshift,
+// finalize: new = (segment sum) / count or old; max shift; master, ch, cn.
+// from_pieces: the segment sum is sums[k] plus the continuation partials of
+// the following pieces (fk_reduce.cu); otherwise sums[k] is complete.
+int launch_finalize(const float *sums, const float *first, int pieces, const int32_t *counts,
+                    const int32_t *offsets, float *centers, void *ch, float *cn, int dtype, int B,
+                    int K, int d, long long Kpad, unsigned *maxshift, bool from_pieces,
                     cudaStream_t s);
+// streamed path: gsum[k] += segment sum of one chunk, gcounts[k] += counts[k].
+int launch_accumulate(const float *sums, const float *first, int pieces, const int32_t *counts,
+                      const int32_t *offsets, int K, int d, float *gsum, int32_t *gcounts,
+                      cudaStream_t s);
 
 int launch_assign_f32(const float *x, const float *c, int B, long long N, int K, int d,
                       int32_t *ids, cudaStream_t s);
 int launch_assign_tc(const void *x, const void *ch, const float *cn, int dtype, int B, long long N,
                      int K, int d, long long Kpad, int32_t *ids, int *err, cudaStream_t s);
 
-// counting sort: counts / offsets optional; keys_out + perm always written.
-// accumulate_counts: add into counts instead of overwriting.
+// counting sort: counts / offsets optional (workspace offsets are used when
+// NULL); perm always written, keys_out (sorted ids) when not NULL.
 int run_sort(Workspace *ws, const int32_t *ids, int B, long long N, int K, int32_t *counts,
-             int32_t *offsets, int32_t *perm, int32_t *keys_out, bool accumulate_counts,
-             cudaStream_t s);
+             int32_t *offsets, int32_t *perm, int32_t *keys_out, cudaStream_t s);
 
+// segment reduce: owner partials to sums (B, K, d), continuation partials to
+// first (B, pieces_of(N), d).
 int launch_segreduce(const void *x, int dtype, const int32_t *skeys, const int32_t *perm, int B,
-                     long long N, int K, int d, float *sums, cudaStream_t s);
+                     long long N, int K, int d, float *sums, float *first, cudaStream_t s);
 
 }  // namespace fk
