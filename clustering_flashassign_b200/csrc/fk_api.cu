@@ -49,6 +49,9 @@ int read_device_error(Workspace *ws, cudaStream_t s) {
   FK_CUDA(cudaMemsetAsync(ws->err, 0, sizeof(int), s));
   FK_CUDA(cudaStreamSynchronize(s));
   if (h == DEV_TIMEOUT) return set_error(FK_ETIMEOUT, "a kernel's bounded wait expired");
+  if (h == DEV_RANGE)
+    return set_error(FK_EUNSUPPORTED,
+                     "a squared norm reached 2^32, beyond the fp16 tensor-core norm digits");
   return set_error(FK_EINVAL, "an id outside [0, K) reached the update");
 }
 
@@ -65,10 +68,10 @@ int prepare_update(Workspace *ws, int B, long long n, int K, int d) {
   return FK_OK;
 }
 
-// Steps a2-a5 on device-resident points; ch / cn (nullable) receive the dtype
-// copy and ||c||^2 of the new centroids for the next assign.
+// Steps a2-a5 on device-resident points; ch / cnx (nullable) receive the dtype
+// copy and the tensor-core extension rows of the new centroids for the next assign.
 int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long N, int K, int d,
-              int dtype, float *centers, int32_t *counts_out, void *ch, float *cn, long long Kpad,
+              int dtype, float *centers, int32_t *counts_out, void *ch, void *cnx, long long Kpad,
               cudaStream_t s) {
   note_update_call();
   int32_t *counts = counts_out;
@@ -90,16 +93,16 @@ int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long
     FK_TRY(launch_segreduce(x, dtype, keys, perm, B, N, K, d, sums, first, s));
   }
   PhaseTimer t(PH_FINALIZE, s);
-  return launch_finalize(sums, first, pieces_of(N), counts, offsets, centers, ch, cn, dtype, B, K,
-                         d, Kpad, ws->maxshift, true, s);
+  return launch_finalize(sums, first, pieces_of(N), counts, offsets, centers, ch, cnx, dtype, B, K,
+                         d, Kpad, ws->maxshift, true, ws->err, s);
 }
 
-int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const float *cn, int B,
-                       long long N, int K, int d, int dtype, long long Kpad, int32_t *ids,
-                       cudaStream_t s) {
+int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const void *cnx,
+                       const float *xn, int B, long long N, int K, int d, int dtype, long long Kpad,
+                       int32_t *ids, cudaStream_t s) {
   PhaseTimer t(PH_ASSIGN, s);
   if (dtype == FK_F32) return launch_assign_f32((const float *)x, (const float *)cdt, B, N, K, d, ids, s);
-  return launch_assign_tc(x, cdt, cn, dtype, B, N, K, d, Kpad, ids, ws->err, s);
+  return launch_assign_tc(x, cdt, cnx, xn, dtype, B, N, K, d, Kpad, ids, ws->err, s);
 }
 
 int read_shift(Workspace *ws, cudaStream_t s, float *out) {
@@ -139,12 +142,12 @@ int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void
   FK_TRY(ensure_copy_engine(ws));
   for (int i = 0; i < 2; ++i) FK_TRY(ensure(ws->chunk[i], (size_t)chunk * d * es));
   void *ch = nullptr;
-  float *cn = nullptr;
+  char *cnx = nullptr;
   if (dtype != FK_F32) {
     FK_TRY(ensure(ws->ch, (size_t)B * K * d * es));
-    FK_TRY(ensure(ws->cn, (size_t)B * Kpad * sizeof(float)));
+    FK_TRY(ensure(ws->cn, ext_bytes(B, Kpad)));
     ch = ws->ch.p;
-    cn = (float *)ws->cn.p;
+    cnx = (char *)ws->cn.p;
   }
   // per chunk: counts, offsets, owner / continuation partials (one batch);
   // per iteration: running sums and counts of every batch
@@ -153,7 +156,7 @@ int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void
   FK_TRY(ensure(ws->gcounts, (size_t)B * K * sizeof(int32_t)));
   int32_t *counts = (int32_t *)ws->counts.p, *gcounts = (int32_t *)ws->gcounts.p;
   float *gsum = (float *)ws->gsum.p;
-  FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cn, s));
+  FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cnx, ws->err, s));
   FK_TRY(prepare_update(ws, 1, chunk, K, d));
   float *sums = (float *)ws->sums.p, *first = (float *)ws->first.p;
   int32_t *keys = (int32_t *)ws->keys_a.p, *perm = (int32_t *)ws->vals_a.p;
@@ -179,7 +182,7 @@ int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void
         int32_t *idc = ids_dev + (size_t)b * N + n0;
         const void *cb = dtype == FK_F32 ? (const void *)(cen_dev + (size_t)b * K * d)
                                          : (const void *)((const char *)ch + (size_t)b * K * d * es);
-        FK_TRY(do_assign_resident(ws, xb, cb, cn ? cn + (size_t)b * Kpad : nullptr, 1, nc, K, d, dtype,
+        FK_TRY(do_assign_resident(ws, xb, cb, cnx ? cnx + ext_bytes(b, Kpad) : nullptr, nullptr, 1, nc, K, d, dtype,
                                   Kpad, idc, s));
         {
           PhaseTimer t(PH_SORT, s);
@@ -196,8 +199,8 @@ int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void
     }
     {
       PhaseTimer t(PH_FINALIZE, s);
-      FK_TRY(launch_finalize(gsum, nullptr, 0, gcounts, nullptr, cen_dev, ch, cn, dtype, B, K, d,
-                             Kpad, ws->maxshift, false, s));
+      FK_TRY(launch_finalize(gsum, nullptr, 0, gcounts, nullptr, cen_dev, ch, cnx, dtype, B, K, d,
+                             Kpad, ws->maxshift, false, ws->err, s));
     }
     if (tol > 0.f || verbose) {
       float ms = 0.f;
@@ -231,13 +234,13 @@ int fk_assign(const void *x, const void *c, int B, long long N, int K, int d, in
   Workspace *ws;
   FK_TRY(workspace_for(s, &ws));
   const long long Kpad = kpad_of(K);
-  float *cn = nullptr;
+  void *cnx = nullptr;
   if (tc) {
-    FK_TRY(ensure(ws->cn, (size_t)B * Kpad * sizeof(float)));
-    cn = (float *)ws->cn.p;
-    FK_TRY(launch_prep_cn(c, dtype, B, K, d, Kpad, cn, s));
+    FK_TRY(ensure(ws->cn, ext_bytes(B, Kpad)));
+    cnx = ws->cn.p;
+    FK_TRY(launch_prep_cn(c, dtype, B, K, d, Kpad, cnx, ws->err, s));
   }
-  return do_assign_resident(ws, x, c, cn, B, N, K, d, dtype, Kpad, ids, s);
+  return do_assign_resident(ws, x, c, cnx, nullptr, B, N, K, d, dtype, Kpad, ids, s);
 }
 
 int fk_update(const void *x, const int32_t *ids, int B, long long N, int K, int d, float *centers,
@@ -330,18 +333,26 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
   }
   if (!streamed) {
     void *ch = nullptr;
-    float *cn = nullptr;
+    void *cnx = nullptr;
+    float *xn = nullptr;
     if (dtype != FK_F32) {
       FK_TRY(ensure(ws->ch, cbytes));
-      FK_TRY(ensure(ws->cn, (size_t)B * Kpad * sizeof(float)));
+      FK_TRY(ensure(ws->cn, ext_bytes(B, Kpad)));
       ch = ws->ch.p;
-      cn = (float *)ws->cn.p;
+      cnx = ws->cn.p;
+      if (max_iter > 1 && d <= 2 * kBlockK) {
+        // the resident-tile assign ranks with ||x||^2 too; the points do not
+        // change, so their norms are computed once per call
+        FK_TRY(ensure(ws->xn, (size_t)B * N * sizeof(float)));
+        xn = (float *)ws->xn.p;
+        FK_TRY(launch_point_norms(xdev, dtype, (long long)B * N, d, xn, s));
+      }
     }
-    FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cn, s));
+    FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cnx, ws->err, s));
     const void *cassign = dtype == FK_F32 ? (const void *)cen_dev : ch;
     for (int it = 0; it < max_iter; ++it) {
-      FK_TRY(do_assign_resident(ws, xdev, cassign, cn, B, N, K, d, dtype, Kpad, ids_dev, s));
-      FK_TRY(do_update(ws, xdev, ids_dev, B, N, K, d, dtype, cen_dev, nullptr, ch, cn, Kpad, s));
+      FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, ids_dev, s));
+      FK_TRY(do_update(ws, xdev, ids_dev, B, N, K, d, dtype, cen_dev, nullptr, ch, cnx, Kpad, s));
       iters = it + 1;
       if (tol > 0.f || o.verbose) {
         float ms = 0.f;

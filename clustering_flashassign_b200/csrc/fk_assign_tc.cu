@@ -1,39 +1,53 @@
 // FlashAssign on sm_100a tensor cores (step a1 for fp16 / bf16 inputs).
 //
-// ids[b,i] = argmin_k ( ||c_k||^2 - 2 x_i . c_k ), fp32 accumulation, lowest
-// k on ties, without ever writing the (B, N, K) distance matrix
-// ("Flash-KMeans: Fast and Memory-Efficient Exact K-Means", Abstract: the
-// distance computation is fused with an online argmin; "flash-kmeans and the
-// return of exact K-Means on the GPU", section "The point of the kernel is
-// that the distance matrix never exists": point tiles and centroid chunks are
-// streamed on chip and the cross term never leaves it).
+// ids[b,i] = argmin_k ||x_i - c_k||^2, fp32 accumulation, lowest k on ties,
+// without ever writing the (B, N, K) distance matrix ("Flash-KMeans: Fast and
+// Memory-Efficient Exact K-Means", Abstract: the distance computation is fused
+// with an online argmin; "flash-kmeans and the return of exact K-Means on the
+// GPU", section "The point of the kernel is that the distance matrix never
+// exists": point tiles and centroid chunks are streamed on chip and the cross
+// term never leaves it).
 //
-// Mapping on a B200 SM (one persistent CTA per SM, 320 threads):
-//   warp 0      TMA producer: point tiles (128 x d) and centroid chunks
-//               (256 x 64 K-blocks) into 128-byte-swizzled shared memory,
+// Mapping on a B200 SM (one persistent CTA per SM, 352 threads):
+//   warp 0      TMA producer: point tiles (128 x d), centroid chunks (256 x 64
+//               K-blocks) into 128-byte-swizzled shared memory, and each
+//               chunk's norm rows (256 x 16, 32-byte swizzle),
 //   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16, kind::f16)
 //               into a TMEM accumulator; two accumulators (2 x 256 columns =
 //               all 512 TMEM columns) let the MMA of chunk c+1 overlap the
-//               epilogue of chunk c,
-//   warps 2..9  epilogue: tcgen05.ld the 128 x 256 cross-term tile, add
-//               ||c||^2 (v = cn - 2 acc, one FFMA), keep a running
-//               (min, argmin) per point.  Two warps share each TMEM lane
-//               quadrant and split the chunk's columns; their results are
-//               combined once per point tile.
+//               epilogue of chunk c.  After the d loop of a chunk one more
+//               K = 16 step multiplies the point and centroid norm rows
+//               (fk_norms.cuh), so the accumulator already holds the ranking
+//               value and the epilogue reads nothing but TMEM,
+//   warps 2..9  epilogue: tcgen05.ld the 128 x 256 tile and keep a running
+//               argmax per point.  Two warps share each TMEM lane quadrant
+//               and split the chunk's columns; their results are combined
+//               once per point tile,
+//   warp 10     (resident variant) ||x||^2 of each point tile from the shared
+//               copy, written as the tile's norm rows.
 // Two variants, picked by d:
 //   resident X (d <= 128): the point tile stays in shared memory for all K
 //               chunks (double-buffered across tiles); only centroids stream.
+//               acc = -(||x - c||^2 + 2^-10 ||x||^2) / 2 - 2^-14 < 0, so the
+//               epilogue packs the column into the low 7 mantissa bits of acc
+//               (one LOP3 per value) and keeps a three-input float max (half
+//               an instruction per value).  Columns whose acc agree in all
+//               other bits count as tied and the lowest column wins; that
+//               merges values within 2^-16 of each other (relative).
 //   split-d     (d > 128): each pipeline stage carries a 64-wide slice of the
 //               point tile and the matching centroid slice; the d loop runs
 //               inside each K chunk (the pages' split-D path, "flash-kmeans
-//               and the return of exact K-Means on the GPU", section "The point
-//               of the kernel ..." and "Unknown GPUs get a conservative
-//               fallback").  The threshold is set by the shared-memory budget
-//               of this design, not the pages' 512.
-// Rows past N and centroid rows past K are zero-filled by TMA; padded
-// centroid columns carry cn = +inf so they never win.
+//               and the return of exact K-Means on the GPU", sections "The
+//               point of the kernel ..." and "Unknown GPUs get a conservative
+//               fallback").  acc = x.c - ||c||^2 / 2 and the epilogue keeps an
+//               exact (value, column) argmax; its cost is spread over d / 64
+//               K-blocks.  The threshold is set by the shared-memory budget of
+//               this design, not the pages' 512.
+// Rows past N and centroid rows past K are zero-filled by TMA; padded centroid
+// columns carry a sentinel norm row (acc about -2^31 or below) so they never win.
 #include <cuda.h>
 
+#include "fk_norms.cuh"
 #include "fk_sm100.cuh"
 
 namespace fk {
@@ -42,10 +56,15 @@ namespace {
 using namespace sm100;
 
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + kEpiWarps * 32;
+constexpr int kNormWarp = 2 + kEpiWarps;
+constexpr int kThreads = 32 * (kNormWarp + 1);
 constexpr uint32_t kXBlockBytes = kTileM * kBlockK * 2;   // 16 KB
 constexpr uint32_t kCBlockBytes = kChunkN * kBlockK * 2;  // 32 KB
+constexpr uint32_t kAExtBytes = kTileM * kExt * 2;        // 4 KB of point norm rows
+constexpr uint32_t kBExtBytes = kChunkN * kExt * 2;       // 8 KB of centroid norm rows
+constexpr int kExtSlots = 2;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kKeyMask = 0xFFFFFF80u;  // packed keys: 7 column bits
 
 struct TcArgs {
   int N;
@@ -53,8 +72,7 @@ struct TcArgs {
   int total_tiles;
   int nchunks;
   int kblocks;
-  long long Kpad;
-  const float *cn;
+  const float *xn;  // ||x||^2 per point (B, N), or NULL: computed from the shared tile
   int32_t *ids;
   int *err;
   uint32_t idesc;
@@ -63,16 +81,20 @@ struct TcArgs {
 template <bool RESIDENT, int KB, int STAGES>
 struct Layout {
   static constexpr uint32_t kXBytes = RESIDENT ? 2u * KB * kXBlockBytes : 0u;
+  static constexpr uint32_t kAExtOff = kXBytes;
+  static constexpr uint32_t kAExtTotal = RESIDENT ? 2u * kAExtBytes : kAExtBytes;
+  static constexpr uint32_t kBExtOff = kAExtOff + kAExtTotal;
+  static constexpr uint32_t kStagesOff = kBExtOff + kExtSlots * kBExtBytes;
   static constexpr uint32_t kStageBytes = RESIDENT ? kCBlockBytes : kXBlockBytes + kCBlockBytes;
-  static constexpr uint32_t kStagesOff = kXBytes;
   static constexpr uint32_t kBarOff = kStagesOff + STAGES * kStageBytes;
-  // barriers: full[S], empty[S], xfull[2], xempty[2], accfull[2], accempty[2],
-  //           mfull[2], mempty[2], drain
-  static constexpr int kNumBars = 2 * STAGES + 13;
-  static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;       // tmem slot, abort flag
+  // barriers: full[S], empty[S], efull[E], eempty[E], xfull[2], xempty[2],
+  //           xnfull[2], accfull[2], accempty[2], mfull[2], mempty[2], drain
+  static constexpr int kNumBars = 2 * STAGES + 2 * kExtSlots + 15;
+  static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag
   static constexpr uint32_t kMergeOff = (kMiscOff + 16 + 15) / 16 * 16;
   static constexpr uint32_t kBytes = kMergeOff + 2 * kTileM * 8;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+  static_assert(kStagesOff % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
@@ -98,26 +120,104 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return r != 0;
 }
 
-template <bool RESIDENT, int KB, int STAGES>
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed key of one accumulator value: acc < 0 with its low 7 mantissa bits
+// replaced by the column.  For negative floats a larger key means a smaller
+// |acc|, and among equal upper bits the smaller column.
+__device__ __forceinline__ float pack_key(uint32_t acc_bits, uint32_t col) {
+  return __uint_as_float((acc_bits & kKeyMask) | col);
+}
+
+__device__ __forceinline__ float key_hi(float key) {
+  return __uint_as_float(__float_as_uint(key) & kKeyMask);
+}
+
+// Stores one 16-element norm row at row r of a K-major 32-byte-swizzled tile:
+// 16-byte chunk q of row r sits at r * 32 + ((q ^ ((r >> 2) & 1)) * 16).
+template <typename T>
+__device__ __forceinline__ void store_ext_row_sw32(uint8_t *tile, int r, const T (&row)[kExt]) {
+  const int flip = (r >> 2) & 1;
+  uint4 *p = reinterpret_cast<uint4 *>(tile + r * 32);
+  p[flip] = *reinterpret_cast<const uint4 *>(&row[0]);
+  p[flip ^ 1] = *reinterpret_cast<const uint4 *>(&row[8]);
+}
+
+// a0 += lo(v)^2, a1 += hi(v)^2 for two packed 16-bit values, fp32 accumulation
+// (mixed-precision FMA: the 16-bit inputs are exact in fp32, one rounding).
+template <typename T> __device__ __forceinline__ void sq2_acc(uint32_t v, float &a0, float &a1);
+template <> __device__ __forceinline__ void sq2_acc<__half>(uint32_t v, float &a0, float &a1) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "fma.rn.f32.f16 %0, lo, lo, %0;\n\tfma.rn.f32.f16 %1, hi, hi, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(v));
+}
+template <> __device__ __forceinline__ void sq2_acc<__nv_bfloat16>(uint32_t v, float &a0, float &a1) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, lo, lo, %0;\n\tfma.rn.f32.bf16 %1, hi, hi, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(v));
+}
+
+// Running argmax over one 32-column TMEM load, packed keys, four max chains.
+__device__ __forceinline__ void scan_packed(const uint32_t (&r)[32], const uint32_t cb, float &m0,
+                                            float &m1, float &m2, float &m3) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 8) {
+    m0 = max3f(m0, pack_key(r[j + 0], cb + j + 0), pack_key(r[j + 1], cb + j + 1));
+    m1 = max3f(m1, pack_key(r[j + 2], cb + j + 2), pack_key(r[j + 3], cb + j + 3));
+    m2 = max3f(m2, pack_key(r[j + 4], cb + j + 4), pack_key(r[j + 5], cb + j + 5));
+    m3 = max3f(m3, pack_key(r[j + 6], cb + j + 6), pack_key(r[j + 7], cb + j + 7));
+  }
+}
+
+// Exact running argmax over one 32-column TMEM load: chain t sees columns
+// j = t (mod 4) in increasing order and moves only on a strictly larger value.
+__device__ __forceinline__ void scan_exact(const uint32_t (&r)[32], const int cb, float (&lb)[4],
+                                           int (&li)[4]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float v = __uint_as_float(r[j + t]);
+      if (v > lb[t]) {
+        lb[t] = v;
+        li[t] = cb + j + t;
+      }
+    }
+  }
+}
+
+template <typename T, bool RESIDENT, int KB, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     k_flash_assign(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmc,
-                   const TcArgs a) {
+                   const __grid_constant__ CUtensorMap tme, const TcArgs a) {
   using L = Layout<RESIDENT, KB, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const uint32_t x_base = sb;
+  const uint32_t aext_base = sb + L::kAExtOff;
+  const uint32_t bext_base = sb + L::kBExtOff;
   const uint32_t st_base = sb + L::kStagesOff;
   const uint32_t bar0 = sb + L::kBarOff;
+  constexpr int kB2 = 2 * STAGES + 2 * kExtSlots;
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto xfull = [&](int i) { return bar0 + 8u * (2 * STAGES + i); };
-  auto xempty = [&](int i) { return bar0 + 8u * (2 * STAGES + 2 + i); };
-  auto accfull = [&](int i) { return bar0 + 8u * (2 * STAGES + 4 + i); };
-  auto accempty = [&](int i) { return bar0 + 8u * (2 * STAGES + 6 + i); };
-  auto mfull = [&](int i) { return bar0 + 8u * (2 * STAGES + 8 + i); };
-  auto mempty = [&](int i) { return bar0 + 8u * (2 * STAGES + 10 + i); };
-  const uint32_t drain = bar0 + 8u * (2 * STAGES + 12);
+  auto efull = [&](int e) { return bar0 + 8u * (2 * STAGES + e); };
+  auto eempty = [&](int e) { return bar0 + 8u * (2 * STAGES + kExtSlots + e); };
+  auto xfull = [&](int i) { return bar0 + 8u * (kB2 + i); };
+  auto xempty = [&](int i) { return bar0 + 8u * (kB2 + 2 + i); };
+  auto xnfull = [&](int i) { return bar0 + 8u * (kB2 + 4 + i); };
+  auto accfull = [&](int i) { return bar0 + 8u * (kB2 + 6 + i); };
+  auto accempty = [&](int i) { return bar0 + 8u * (kB2 + 8 + i); };
+  auto mfull = [&](int i) { return bar0 + 8u * (kB2 + 10 + i); };
+  auto mempty = [&](int i) { return bar0 + 8u * (kB2 + 12 + i); };
+  const uint32_t drain = bar0 + 8u * (kB2 + 14);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   float2 *merge = reinterpret_cast<float2 *>(smem + L::kMergeOff);
@@ -129,9 +229,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
     }
+    for (int e = 0; e < kExtSlots; ++e) {
+      mbar_init(efull(e), 1);
+      mbar_init(eempty(e), 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(xfull(i), 1);
       mbar_init(xempty(i), 1);
+      mbar_init(xnfull(i), 1);
       mbar_init(accfull(i), 1);
       mbar_init(accempty(i), kEpiWarps);
       mbar_init(mfull(i), kEpiWarps / 2);
@@ -145,10 +250,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmx);
     prefetch_tensormap(&tmc);
+    prefetch_tensormap(&tme);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
+  }
+  if (!RESIDENT && warp == kNormWarp) {
+    // split-d: one constant point-side row (the -S_e that multiply ||c||^2's digits)
+    T row[kExt];
+    ext_point_row<T, false>(0.f, row);
+    for (int r = lane; r < kTileM; r += 32) store_ext_row_sw32<T>(smem + L::kAExtOff, r, row);
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -159,20 +272,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t f = 0, g = 0;
+      uint32_t f = 0, g = 0, e = 0;
       bool ok = true;
+      // Point tiles are loaded one tile ahead: the tile after this one is
+      // requested right after this tile's first chunk, as soon as the MMAs of
+      // the tile before have released its buffer, so the norm warp has a whole
+      // tile of time for it.
+      auto load_x = [&](int tile) -> bool {
+        const int xb = g & 1;
+        if (!mbar_wait(xempty(xb), ((g >> 1) & 1) ^ 1, abort_flag, a.err)) return false;
+        mbar_arrive_expect_tx(xfull(xb), KB * kXBlockBytes);
+        const int b = tile / a.tiles_per_batch;
+        const int row0 = (tile % a.tiles_per_batch) * kTileM;
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_3d(&tmx, x_base + (xb * KB + kb) * kXBlockBytes, xfull(xb), kb * kBlockK, row0, b);
+        ++g;
+        return true;
+      };
+      if (RESIDENT && (int)blockIdx.x < a.total_tiles) ok = load_x(blockIdx.x);
       for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x) {
         const int b = tile / a.tiles_per_batch;
         const int row0 = (tile % a.tiles_per_batch) * kTileM;
-        if (RESIDENT) {
-          const int xb = g & 1;
-          if (!mbar_wait(xempty(xb), ((g >> 1) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
-          mbar_arrive_expect_tx(xfull(xb), KB * kXBlockBytes);
-          for (int kb = 0; kb < KB; ++kb)
-            tma_load_3d(&tmx, x_base + (xb * KB + kb) * kXBlockBytes, xfull(xb), kb * kBlockK, row0, b);
-          ++g;
-        }
         for (int c = 0; ok && c < a.nchunks; ++c) {
+          {  // this chunk's centroid norm rows (used by the chunk's last MMA step)
+            const int es = e % kExtSlots;
+            if (!mbar_wait(eempty(es), ((e / kExtSlots) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+            mbar_arrive_expect_tx(efull(es), kBExtBytes);
+            tma_load_3d(&tme, bext_base + es * kBExtBytes, efull(es), 0, c * kChunkN, b);
+            ++e;
+          }
           for (int kb = 0; kb < kblocks; ++kb) {
             const int s = f % STAGES;
             if (!mbar_wait(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
@@ -187,15 +315,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ++f;
           }
+          if (RESIDENT && ok && c == 0 && tile + (int)gridDim.x < a.total_tiles)
+            ok = load_x(tile + gridDim.x);
         }
       }
-      // tail: make every issued copy and every release of a stage land before exit
+      // tail: make every issued copy and every release of a buffer land before exit
       const bool aborted = *abort_flag != 0;
-      for (uint32_t ff = f > (uint32_t)STAGES ? f - STAGES : 0; ff < f; ++ff) {
-        const int s = ff % STAGES;
-        const uint32_t par = (ff / STAGES) & 1;
-        wait_drain(aborted ? full(s) : empty(s), par, a.err);
-      }
+      for (uint32_t ff = f > (uint32_t)STAGES ? f - STAGES : 0; ff < f; ++ff)
+        wait_drain(aborted ? full(ff % STAGES) : empty(ff % STAGES), (ff / STAGES) & 1, a.err);
+      for (uint32_t ee = e > (uint32_t)kExtSlots ? e - kExtSlots : 0; ee < e; ++ee)
+        wait_drain(aborted ? efull(ee % kExtSlots) : eempty(ee % kExtSlots), (ee / kExtSlots) & 1, a.err);
       if (RESIDENT) {
         for (uint32_t gg = g > 2 ? g - 2 : 0; gg < g; ++gg)
           wait_drain(aborted ? xfull(gg & 1) : xempty(gg & 1), (gg >> 1) & 1, a.err);
@@ -205,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t f = 0, g = 0, h = 0;
+      uint32_t f = 0, g = 0, h = 0, e = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x) {
         int xb = 0;
@@ -214,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(xfull(xb), (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
         }
+        const uint32_t a_ext = aext_base + (RESIDENT ? xb * kAExtBytes : 0u);
         for (int c = 0; ok && c < a.nchunks; ++c) {
           const int ab = h & 1;
           if (!mbar_wait(accempty(ab), ((h >> 1) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
@@ -234,11 +364,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++f;
           }
           if (!ok) break;
+          // the norm step: acc += A_ext . B_ext (fk_norms.cuh)
+          if (RESIDENT && c == 0) {
+            if (!mbar_wait(xnfull(xb), (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+            tc_fence_after();
+          }
+          const int es = e % kExtSlots;
+          if (!mbar_wait(efull(es), (e / kExtSlots) & 1, abort_flag, a.err)) { ok = false; break; }
+          tc_fence_after();
+          mma_f16(d_tmem, desc_k_sw32(a_ext), desc_k_sw32(bext_base + es * kBExtBytes), a.idesc, 1u);
+          mma_commit(eempty(es));
+          ++e;
           mma_commit(accfull(ab));  // accumulator ready for the epilogue
           ++h;
         }
         if (RESIDENT && ok) {
-          mma_commit(xempty(xb));  // point tile no longer needed
+          mma_commit(xempty(xb));  // point tile and its norm rows no longer needed
           ++g;
         }
       }
@@ -246,6 +387,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_drain(drain, 0, a.err);
     }
     __syncwarp();
+  } else if (warp == kNormWarp) {
+    // ------------------------------------------------------------ point norms
+    if (RESIDENT) {
+      uint32_t g = 0;
+      for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++g) {
+        const int xb = g & 1;
+        const int b = tile / a.tiles_per_batch;
+        const int row0 = (tile % a.tiles_per_batch) * kTileM;
+        float xn2[kTileM / 32];
+        if (a.xn) {  // issued before the wait: the loads overlap it
+#pragma unroll
+          for (int q = 0; q < kTileM / 32; ++q) {
+            const int row = row0 + q * 32 + lane;
+            xn2[q] = row < a.N ? __ldg(a.xn + (size_t)b * a.N + row) : 0.f;
+          }
+        }
+        if (!warp_wait(xfull(xb), (g >> 1) & 1, abort_flag, a.err, lane)) break;
+        if (!a.xn) {
+          // lane l sums rows l, l+32, l+64, l+96 of the swizzled tile (16-byte
+          // chunk j of row r sits at chunk j ^ (r & 7); r & 7 == l & 7 here)
+          float s0[kTileM / 32], s1[kTileM / 32];
+#pragma unroll
+          for (int q = 0; q < kTileM / 32; ++q) s0[q] = s1[q] = 0.f;
+#pragma unroll
+          for (int kb = 0; kb < KB; ++kb) {
+            const uint8_t *blk = smem + (xb * KB + kb) * kXBlockBytes + lane * 128;
+#pragma unroll 2
+            for (int j = 0; j < 8; ++j) {
+              const int off = (j ^ (lane & 7)) << 4;
+              uint4 v[kTileM / 32];
+#pragma unroll
+              for (int q = 0; q < kTileM / 32; ++q)
+                v[q] = *reinterpret_cast<const uint4 *>(blk + q * 32 * 128 + off);
+#pragma unroll
+              for (int q = 0; q < kTileM / 32; ++q) {
+                sq2_acc<T>(v[q].x, s0[q], s1[q]);
+                sq2_acc<T>(v[q].y, s0[q], s1[q]);
+                sq2_acc<T>(v[q].z, s0[q], s1[q]);
+                sq2_acc<T>(v[q].w, s0[q], s1[q]);
+              }
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < kTileM / 32; ++q) xn2[q] = s0[q] + s1[q];
+        }
+        bool clamped = false;
+#pragma unroll
+        for (int q = 0; q < kTileM / 32; ++q) {
+          alignas(16) T row[kExt];
+          clamped |= ext_point_row<T, true>(xn2[q], row);
+          store_ext_row_sw32<T>(smem + L::kAExtOff + xb * kAExtBytes, q * 32 + lane, row);
+        }
+        if (clamped) atomicCAS(a.err, DEV_OK, DEV_RANGE);
+        fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xnfull(xb));
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
@@ -258,73 +457,79 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x, ++u) {
       const int b = tile / a.tiles_per_batch;
       const int row0 = (tile % a.tiles_per_batch) * kTileM;
-      const float *cnb = a.cn + (size_t)b * a.Kpad + half * 128;
-      float best = __int_as_float(0x7f800000);
-      int bidx = 0;
+      float best = __int_as_float(0xff800000);  // -inf
+      int bidx = 0;                              // chunk (packed) or column (exact) of best
       for (int c = 0; c < a.nchunks; ++c, ++h) {
         const int ab = h & 1;
         if (!warp_wait(accfull(ab), (h >> 1) & 1, abort_flag, a.err, lane)) { ok = false; break; }
         tc_fence_after();
-        const float *cnc = cnb + (size_t)c * kChunkN;
-        float lb[4] = {best, best, best, best};
-        int li[4] = {-1, -1, -1, -1};
-#pragma unroll
-        for (int gp = 0; gp < 2; ++gp) {
-          uint32_t r0[32], r1[32];
-          tmem_ld_32x32b_x32(t_lane + ab * kChunkN + gp * 64, r0);
-          tmem_ld_32x32b_x32(t_lane + ab * kChunkN + gp * 64 + 32, r1);
+        const uint32_t tb = t_lane + ab * kChunkN;
+        uint32_t ra[32], rb[32], rc[32], rd[32];
+        tmem_ld_32x32b_x32(tb, ra);
+        tmem_ld_32x32b_x32(tb + 32, rb);
+        tmem_wait_ld();
+        tmem_ld_32x32b_x32(tb + 64, rc);  // in flight while ra, rb are scanned
+        tmem_ld_32x32b_x32(tb + 96, rd);
+        if (RESIDENT) {
+          float m0 = best, m1 = best, m2 = best, m3 = best;
+          scan_packed(ra, 0, m0, m1, m2, m3);
+          scan_packed(rb, 32, m0, m1, m2, m3);
           tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            const float4 cv = __ldg(reinterpret_cast<const float4 *>(cnc + gp * 64 + j));
-            const float v0 = fmaf(__uint_as_float(r0[j + 0]), -2.f, cv.x);
-            const float v1 = fmaf(__uint_as_float(r0[j + 1]), -2.f, cv.y);
-            const float v2 = fmaf(__uint_as_float(r0[j + 2]), -2.f, cv.z);
-            const float v3 = fmaf(__uint_as_float(r0[j + 3]), -2.f, cv.w);
-            if (v0 < lb[0]) { lb[0] = v0; li[0] = gp * 64 + j + 0; }
-            if (v1 < lb[1]) { lb[1] = v1; li[1] = gp * 64 + j + 1; }
-            if (v2 < lb[2]) { lb[2] = v2; li[2] = gp * 64 + j + 2; }
-            if (v3 < lb[3]) { lb[3] = v3; li[3] = gp * 64 + j + 3; }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(accempty(ab));  // accumulator may be overwritten
+          scan_packed(rc, 64, m0, m1, m2, m3);
+          scan_packed(rd, 96, m0, m1, m2, m3);
+          const float m = fmaxf(max3f(m0, m1, m2), m3);
+          // a later chunk must beat the running best in the upper bits
+          if (key_hi(m) > key_hi(best)) {
+            best = m;
+            bidx = c;
           }
+        } else {
+          float lb[4] = {best, best, best, best};
+          int li[4] = {-1, -1, -1, -1};
+          scan_exact(ra, 0, lb, li);
+          scan_exact(rb, 32, lb, li);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(accempty(ab));
+          scan_exact(rc, 64, lb, li);
+          scan_exact(rd, 96, lb, li);
+          // merge the four chains: larger value, then lower column
+          float m = lb[0];
+          int mi = li[0];
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            const float4 cv = __ldg(reinterpret_cast<const float4 *>(cnc + gp * 64 + 32 + j));
-            const float v0 = fmaf(__uint_as_float(r1[j + 0]), -2.f, cv.x);
-            const float v1 = fmaf(__uint_as_float(r1[j + 1]), -2.f, cv.y);
-            const float v2 = fmaf(__uint_as_float(r1[j + 2]), -2.f, cv.z);
-            const float v3 = fmaf(__uint_as_float(r1[j + 3]), -2.f, cv.w);
-            if (v0 < lb[0]) { lb[0] = v0; li[0] = gp * 64 + 32 + j + 0; }
-            if (v1 < lb[1]) { lb[1] = v1; li[1] = gp * 64 + 32 + j + 1; }
-            if (v2 < lb[2]) { lb[2] = v2; li[2] = gp * 64 + 32 + j + 2; }
-            if (v3 < lb[3]) { lb[3] = v3; li[3] = gp * 64 + 32 + j + 3; }
+          for (int t = 1; t < 4; ++t) {
+            if (li[t] >= 0 && (mi < 0 || lb[t] > m || (lb[t] == m && li[t] < mi))) {
+              m = lb[t];
+              mi = li[t];
+            }
           }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(accempty(ab));  // accumulator may be overwritten
-        // merge the four chains: smaller value, then lower column
-        float m = lb[0];
-        int mi = li[0];
-#pragma unroll
-        for (int t = 1; t < 4; ++t) {
-          if (li[t] >= 0 && (mi < 0 || lb[t] < m || (lb[t] == m && li[t] < mi))) {
-            m = lb[t];
-            mi = li[t];
+          if (mi >= 0) {  // strictly above the running best (chains start at it)
+            best = m;
+            bidx = c * kChunkN + half * 128 + mi;
           }
-        }
-        if (mi >= 0) {  // strictly below the running best (chains start at it)
-          best = m;
-          bidx = c * kChunkN + half * 128 + mi;
         }
       }
       if (!ok) break;
-      // combine the two column halves of each row: lower value, then lower index
+      float val;
+      int idx;
+      if (RESIDENT) {
+        val = key_hi(best);
+        idx = bidx * kChunkN + half * 128 + (int)(__float_as_uint(best) & ~kKeyMask);
+      } else {
+        val = best;
+        idx = bidx;
+      }
+      // combine the two column halves of each row: larger value, then lower index
       const int p = u & 1;
       const uint32_t vpar = (u >> 1) & 1;
       float2 *slot = merge + p * kTileM + r_in_tile;
       if (half == 1) {
         if (!warp_wait(mempty(p), vpar ^ 1, abort_flag, a.err, lane)) { ok = false; break; }
-        *slot = make_float2(best, __int_as_float(bidx));
+        *slot = make_float2(val, __int_as_float(idx));
         __syncwarp();
         if (lane == 0) mbar_arrive(mfull(p));
       } else {
@@ -332,14 +537,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float2 o = *slot;
         __syncwarp();
         if (lane == 0) mbar_arrive(mempty(p));
-        const float ob = o.x;
+        const float ov = o.x;
         const int oi = __float_as_int(o.y);
-        if (ob < best || (ob == best && oi < bidx)) {
-          best = ob;
-          bidx = oi;
-        }
+        if (ov > val || (ov == val && oi < idx)) idx = oi;
         const int row = row0 + r_in_tile;
-        if (row < a.N) a.ids[(size_t)b * a.N + row] = bidx;
+        if (row < a.N) a.ids[(size_t)b * a.N + row] = idx;
       }
     }
   }
@@ -349,6 +551,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// ||x_i||^2 of every point, one thread per row, summed in exactly the order
+// the norm warp uses on a shared tile (16-byte chunks in order; low halves into
+// s0, high halves into s1; s0 + s1), so both give bit-identical norms and a
+// Lloyd run that precomputes them assigns exactly like fk_assign.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    k_point_norms(const T *__restrict__ x, long long rows, int d, float *__restrict__ xn) {
+  const int chunks = d / 8;
+  for (long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x; r < rows;
+       r += (long long)gridDim.x * blockDim.x) {
+    const uint4 *row = reinterpret_cast<const uint4 *>(x + (size_t)r * d);
+    float s0 = 0.f, s1 = 0.f;
+    for (int j = 0; j < chunks; ++j) {
+      const uint4 v = __ldg(row + j);
+      sq2_acc<T>(v.x, s0, s1);
+      sq2_acc<T>(v.y, s0, s1);
+      sq2_acc<T>(v.z, s0, s1);
+      sq2_acc<T>(v.w, s0, s1);
+    }
+    xn[r] = s0 + s1;
+  }
+}
+
+template <typename T>
+int point_norms_t(const void *x, long long rows, int d, float *xn, cudaStream_t s) {
+  long long blocks = (rows + 255) / 256;
+  const long long cap = (long long)num_sms() * 16;
+  if (blocks > cap) blocks = cap;
+  k_point_norms<T><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const T *>(x), rows, d, xn);
+  count_launch();
+  FK_CUDA(cudaGetLastError());
+  return FK_OK;
 }
 
 // ---------------------------------------------------------------- host side
@@ -372,46 +608,60 @@ int get_encoder(EncodeTiledFn *out) {
   return FK_OK;
 }
 
-// (d, rows, B) tensor of 16-bit elements, box (64, box_rows, 1), 128-byte swizzle.
-int encode_3d(CUtensorMap *map, const void *base, int dtype, int d, long long rows, int B,
-              int box_rows) {
+// (inner, rows, B) tensor of 16-bit elements, box (box_inner, box_rows, 1).
+int encode_3d(CUtensorMap *map, const void *base, int dtype, int inner, long long rows, int B,
+              int box_inner, int box_rows, CUtensorMapSwizzle swz) {
   EncodeTiledFn enc;
   FK_TRY(get_encoder(&enc));
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)B};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
-  cuuint32_t box[3] = {(cuuint32_t)kBlockK, (cuuint32_t)box_rows, 1};
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)rows * inner * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, dtype == FK_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                    3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(FK_ECUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
   return FK_OK;
 }
 
-template <bool RESIDENT, int KB, int STAGES>
-int launch_variant(const CUtensorMap &tmx, const CUtensorMap &tmc, const TcArgs &a, int grid,
-                   cudaStream_t s) {
+template <typename T, bool RESIDENT, int KB, int STAGES>
+int launch_variant(const CUtensorMap &tmx, const CUtensorMap &tmc, const CUtensorMap &tme,
+                   const TcArgs &a, int grid, cudaStream_t s) {
   using L = Layout<RESIDENT, KB, STAGES>;
   static bool attr = false;
   if (!attr) {
-    FK_CUDA(cudaFuncSetAttribute(k_flash_assign<RESIDENT, KB, STAGES>,
+    FK_CUDA(cudaFuncSetAttribute(k_flash_assign<T, RESIDENT, KB, STAGES>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc));
     attr = true;
   }
-  k_flash_assign<RESIDENT, KB, STAGES><<<grid, kThreads, L::kAlloc, s>>>(tmx, tmc, a);
+  k_flash_assign<T, RESIDENT, KB, STAGES><<<grid, kThreads, L::kAlloc, s>>>(tmx, tmc, tme, a);
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
 
+template <typename T>
+int launch_typed(const CUtensorMap &tmx, const CUtensorMap &tmc, const CUtensorMap &tme,
+                 const TcArgs &a, int grid, cudaStream_t s) {
+  if (a.kblocks == 1) return launch_variant<T, true, 1, 5>(tmx, tmc, tme, a, grid, s);
+  if (a.kblocks == 2) return launch_variant<T, true, 2, 4>(tmx, tmc, tme, a, grid, s);
+  return launch_variant<T, false, 1, 4>(tmx, tmc, tme, a, grid, s);
+}
+
 }  // namespace
 
-int launch_assign_tc(const void *x, const void *ch, const float *cn, int dtype, int B, long long N,
-                     int K, int d, long long Kpad, int32_t *ids, int *err, cudaStream_t s) {
-  CUtensorMap tmx, tmc;
-  FK_TRY(encode_3d(&tmx, x, dtype, d, N, B, kTileM));
-  FK_TRY(encode_3d(&tmc, ch, dtype, d, K, B, kChunkN));
+int launch_point_norms(const void *x, int dtype, long long rows, int d, float *xn, cudaStream_t s) {
+  if (dtype == FK_BF16) return point_norms_t<__nv_bfloat16>(x, rows, d, xn, s);
+  return point_norms_t<__half>(x, rows, d, xn, s);
+}
+
+int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float *xn, int dtype,
+                     int B, long long N, int K, int d, long long Kpad, int32_t *ids, int *err,
+                     cudaStream_t s) {
+  CUtensorMap tmx, tmc, tme;
+  FK_TRY(encode_3d(&tmx, x, dtype, d, N, B, kBlockK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B));
+  FK_TRY(encode_3d(&tmc, ch, dtype, d, K, B, kBlockK, kChunkN, CU_TENSOR_MAP_SWIZZLE_128B));
+  FK_TRY(encode_3d(&tme, cnx, dtype, kExt, Kpad, B, kExt, kChunkN, CU_TENSOR_MAP_SWIZZLE_32B));
   TcArgs a;
   a.N = (int)N;
   a.tiles_per_batch = (int)((N + kTileM - 1) / kTileM);
@@ -420,16 +670,14 @@ int launch_assign_tc(const void *x, const void *ch, const float *cn, int dtype, 
   a.total_tiles = (int)total;
   a.nchunks = (K + kChunkN - 1) / kChunkN;
   a.kblocks = (d + kBlockK - 1) / kBlockK;
-  a.Kpad = Kpad;
-  a.cn = cn;
+  a.xn = xn;
   a.ids = ids;
   a.err = err;
   a.idesc = sm100::idesc_f16(dtype == FK_BF16 ? 1u : 0u, kTileM, kChunkN);
   int grid = num_sms();
   if (total < grid) grid = (int)total;
-  if (a.kblocks == 1) return launch_variant<true, 1, 5>(tmx, tmc, a, grid, s);
-  if (a.kblocks == 2) return launch_variant<true, 2, 4>(tmx, tmc, a, grid, s);
-  return launch_variant<false, 1, 4>(tmx, tmc, a, grid, s);
+  if (dtype == FK_BF16) return launch_typed<__nv_bfloat16>(tmx, tmc, tme, a, grid, s);
+  return launch_typed<__half>(tmx, tmc, tme, a, grid, s);
 }
 
 }  // namespace fk

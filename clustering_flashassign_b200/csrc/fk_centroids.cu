@@ -18,6 +18,7 @@
 #include <cuda_fp16.h>
 
 #include "fk_internal.h"
+#include "fk_norms.cuh"
 
 namespace fk {
 namespace {
@@ -39,7 +40,22 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 constexpr int kWarpsPerBlock = 8;
-constexpr float kInf = __builtin_huge_valf();
+
+// Writes the tensor-core extension row of one centroid (see fk_norms.cuh);
+// rows past K get the sentinel row.  A norm beyond the fp16 digits' range is
+// recorded as DEV_RANGE in the device error word.
+template <typename T>
+__device__ __forceinline__ void store_ext(T *cnx, long long w, bool real, float cn, int *err) {
+  if constexpr (sizeof(T) == 2) {
+    alignas(16) T row[kExt];
+    if (ext_centroid_row<T>(cn, real, row) && err) atomicCAS(err, DEV_OK, DEV_RANGE);
+    uint4 *dst = reinterpret_cast<uint4 *>(cnx + (size_t)w * kExt);
+    dst[0] = *reinterpret_cast<const uint4 *>(&row[0]);
+    dst[1] = *reinterpret_cast<const uint4 *>(&row[8]);
+  } else {
+    (void)cnx; (void)w; (void)real; (void)cn; (void)err;
+  }
+}
 
 // Element loop shared by every kernel: f(j, n) handles elements j .. j+n-1.
 template <bool V4, typename F>
@@ -53,13 +69,13 @@ __device__ __forceinline__ void for_lane_elems(int d, int lane, F &&f) {
 
 template <typename T, bool V4>
 __global__ void k_prep_cn(const T *__restrict__ c, int B, int K, int d, long long Kpad,
-                          float *__restrict__ cn) {
+                          T *__restrict__ cnx, int *err) {
   const long long w = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= (long long)B * Kpad) return;
   const int b = (int)(w / Kpad), k = (int)(w % Kpad);
   if (k >= K) {
-    if (lane == 0) cn[w] = kInf;  // padded columns never win
+    if (lane == 0) store_ext<T>(cnx, w, false, 0.f, err);
     return;
   }
   const T *row = c + ((size_t)b * K + k) * d;
@@ -71,18 +87,19 @@ __global__ void k_prep_cn(const T *__restrict__ c, int B, int K, int d, long lon
     }
   });
   s = warp_sum(s);
-  if (lane == 0) cn[w] = s;
+  if (lane == 0) store_ext<T>(cnx, w, true, s, err);
 }
 
 template <typename T, bool V4>
 __global__ void k_init(const T *__restrict__ init, int B, int K, int d, long long Kpad,
-                       float *__restrict__ master, T *__restrict__ ch, float *__restrict__ cn) {
+                       float *__restrict__ master, T *__restrict__ ch, T *__restrict__ cnx,
+                       int *err) {
   const long long w = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= (long long)B * Kpad) return;
   const int b = (int)(w / Kpad), k = (int)(w % Kpad);
   if (k >= K) {
-    if (lane == 0 && cn) cn[w] = kInf;
+    if (lane == 0 && cnx) store_ext<T>(cnx, w, false, 0.f, err);
     return;
   }
   const size_t off = ((size_t)b * K + k) * d;
@@ -97,7 +114,7 @@ __global__ void k_init(const T *__restrict__ init, int B, int K, int d, long lon
     }
   });
   s = warp_sum(s);
-  if (lane == 0 && cn) cn[w] = s;
+  if (lane == 0 && cnx) store_ext<T>(cnx, w, true, s, err);
 }
 
 // Sum of cluster w: the owner piece's partial plus the continuation partials
@@ -115,8 +132,8 @@ template <typename T, bool V4, bool FROM_PIECES>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     k_finalize(const float *__restrict__ sums, const float *__restrict__ first, int pieces,
                const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets,
-               float *__restrict__ centers, T *__restrict__ ch, float *__restrict__ cn, int B, int K,
-               int d, long long Kpad, unsigned *__restrict__ maxshift) {
+               float *__restrict__ centers, T *__restrict__ ch, T *__restrict__ cnx, int B, int K,
+               int d, long long Kpad, unsigned *__restrict__ maxshift, int *err) {
   __shared__ float wmax[kWarpsPerBlock];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float my_max = 0.f;
@@ -151,7 +168,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     });
     shift2 = warp_sum(shift2);
     nrm = warp_sum(nrm);
-    if (lane == 0 && cn) cn[(size_t)b * Kpad + k] = nrm;
+    if (lane == 0 && cnx) store_ext<T>(cnx, (long long)b * Kpad + k, true, nrm, err);
     my_max = fmaxf(my_max, sqrtf(shift2));
   }
   if (lane == 0) wmax[warp] = my_max;
@@ -192,10 +209,10 @@ inline unsigned blocks_for(long long warps) {
 }
 
 template <typename T>
-int prep_t(const void *c, int B, int K, int d, long long Kpad, float *cn, cudaStream_t s) {
+int prep_t(const void *c, int B, int K, int d, long long Kpad, void *cnx, int *err, cudaStream_t s) {
   const unsigned g = blocks_for((long long)B * Kpad);
-  if (d % 4 == 0) k_prep_cn<T, true><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)c, B, K, d, Kpad, cn);
-  else k_prep_cn<T, false><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)c, B, K, d, Kpad, cn);
+  if (d % 4 == 0) k_prep_cn<T, true><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)c, B, K, d, Kpad, (T *)cnx, err);
+  else k_prep_cn<T, false><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)c, B, K, d, Kpad, (T *)cnx, err);
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;
@@ -203,12 +220,12 @@ int prep_t(const void *c, int B, int K, int d, long long Kpad, float *cn, cudaSt
 
 template <typename T>
 int init_t(const void *init, int B, int K, int d, long long Kpad, float *master, void *ch,
-           float *cn, cudaStream_t s) {
+           void *cnx, int *err, cudaStream_t s) {
   const unsigned g = blocks_for((long long)B * Kpad);
   if (d % 4 == 0)
-    k_init<T, true><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)init, B, K, d, Kpad, master, (T *)ch, cn);
+    k_init<T, true><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)init, B, K, d, Kpad, master, (T *)ch, (T *)cnx, err);
   else
-    k_init<T, false><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)init, B, K, d, Kpad, master, (T *)ch, cn);
+    k_init<T, false><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)init, B, K, d, Kpad, master, (T *)ch, (T *)cnx, err);
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;
@@ -216,17 +233,17 @@ int init_t(const void *init, int B, int K, int d, long long Kpad, float *master,
 
 template <typename T, bool FP>
 int fin_t(const float *sums, const float *first, int pieces, const int32_t *counts,
-          const int32_t *offsets, float *centers, void *ch, float *cn, int B, int K, int d,
-          long long Kpad, unsigned *maxshift, cudaStream_t s) {
+          const int32_t *offsets, float *centers, void *ch, void *cnx, int B, int K, int d,
+          long long Kpad, unsigned *maxshift, int *err, cudaStream_t s) {
   unsigned g = blocks_for((long long)B * K);
   const unsigned cap = (unsigned)num_sms() * 8;
   if (g > cap) g = cap;
   if (d % 4 == 0)
     k_finalize<T, true, FP><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, centers,
-                                                              (T *)ch, cn, B, K, d, Kpad, maxshift);
+                                                              (T *)ch, (T *)cnx, B, K, d, Kpad, maxshift, err);
   else
     k_finalize<T, false, FP><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, centers,
-                                                               (T *)ch, cn, B, K, d, Kpad, maxshift);
+                                                               (T *)ch, (T *)cnx, B, K, d, Kpad, maxshift, err);
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;
@@ -234,32 +251,32 @@ int fin_t(const float *sums, const float *first, int pieces, const int32_t *coun
 
 }  // namespace
 
-int launch_prep_cn(const void *c, int dtype, int B, int K, int d, long long Kpad, float *cn,
-                   cudaStream_t s) {
-  if (dtype == FK_F16) return prep_t<__half>(c, B, K, d, Kpad, cn, s);
-  if (dtype == FK_BF16) return prep_t<__nv_bfloat16>(c, B, K, d, Kpad, cn, s);
-  return prep_t<float>(c, B, K, d, Kpad, cn, s);
+int launch_prep_cn(const void *c, int dtype, int B, int K, int d, long long Kpad, void *cnx,
+                   int *err, cudaStream_t s) {
+  if (dtype == FK_F16) return prep_t<__half>(c, B, K, d, Kpad, cnx, err, s);
+  if (dtype == FK_BF16) return prep_t<__nv_bfloat16>(c, B, K, d, Kpad, cnx, err, s);
+  return prep_t<float>(c, B, K, d, Kpad, cnx, err, s);
 }
 
 int launch_init_centers(const void *init, int dtype, int B, int K, int d, long long Kpad,
-                        float *master, void *ch, float *cn, cudaStream_t s) {
-  if (dtype == FK_F16) return init_t<__half>(init, B, K, d, Kpad, master, ch, cn, s);
-  if (dtype == FK_BF16) return init_t<__nv_bfloat16>(init, B, K, d, Kpad, master, ch, cn, s);
-  return init_t<float>(init, B, K, d, Kpad, master, nullptr, cn, s);
+                        float *master, void *ch, void *cnx, int *err, cudaStream_t s) {
+  if (dtype == FK_F16) return init_t<__half>(init, B, K, d, Kpad, master, ch, cnx, err, s);
+  if (dtype == FK_BF16) return init_t<__nv_bfloat16>(init, B, K, d, Kpad, master, ch, cnx, err, s);
+  return init_t<float>(init, B, K, d, Kpad, master, nullptr, nullptr, err, s);
 }
 
 int launch_finalize(const float *sums, const float *first, int pieces, const int32_t *counts,
-                    const int32_t *offsets, float *centers, void *ch, float *cn, int dtype, int B,
-                    int K, int d, long long Kpad, unsigned *maxshift, bool from_pieces,
+                    const int32_t *offsets, float *centers, void *ch, void *cnx, int dtype, int B,
+                    int K, int d, long long Kpad, unsigned *maxshift, bool from_pieces, int *err,
                     cudaStream_t s) {
   if (dtype == FK_F16)
-    return from_pieces ? fin_t<__half, true>(sums, first, pieces, counts, offsets, centers, ch, cn, B, K, d, Kpad, maxshift, s)
-                       : fin_t<__half, false>(sums, first, pieces, counts, offsets, centers, ch, cn, B, K, d, Kpad, maxshift, s);
+    return from_pieces ? fin_t<__half, true>(sums, first, pieces, counts, offsets, centers, ch, cnx, B, K, d, Kpad, maxshift, err, s)
+                       : fin_t<__half, false>(sums, first, pieces, counts, offsets, centers, ch, cnx, B, K, d, Kpad, maxshift, err, s);
   if (dtype == FK_BF16)
-    return from_pieces ? fin_t<__nv_bfloat16, true>(sums, first, pieces, counts, offsets, centers, ch, cn, B, K, d, Kpad, maxshift, s)
-                       : fin_t<__nv_bfloat16, false>(sums, first, pieces, counts, offsets, centers, ch, cn, B, K, d, Kpad, maxshift, s);
-  return from_pieces ? fin_t<float, true>(sums, first, pieces, counts, offsets, centers, nullptr, cn, B, K, d, Kpad, maxshift, s)
-                     : fin_t<float, false>(sums, first, pieces, counts, offsets, centers, nullptr, cn, B, K, d, Kpad, maxshift, s);
+    return from_pieces ? fin_t<__nv_bfloat16, true>(sums, first, pieces, counts, offsets, centers, ch, cnx, B, K, d, Kpad, maxshift, err, s)
+                       : fin_t<__nv_bfloat16, false>(sums, first, pieces, counts, offsets, centers, ch, cnx, B, K, d, Kpad, maxshift, err, s);
+  return from_pieces ? fin_t<float, true>(sums, first, pieces, counts, offsets, centers, nullptr, nullptr, B, K, d, Kpad, maxshift, err, s)
+                     : fin_t<float, false>(sums, first, pieces, counts, offsets, centers, nullptr, nullptr, B, K, d, Kpad, maxshift, err, s);
 }
 
 int launch_accumulate(const float *sums, const float *first, int pieces, const int32_t *counts,

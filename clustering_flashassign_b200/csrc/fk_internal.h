@@ -12,7 +12,9 @@
 namespace fk {
 
 // Device error word values (written by kernels, read by fk_device_error).
-enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_ID = 2 };
+// DEV_RANGE: a squared norm beyond the range of the fp16 norm digits that
+// the tensor-core assign folds into its MMA (||v||^2 >= 2^32).
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_ID = 2, DEV_RANGE = 3 };
 
 // Bounded waits inside kernels give up after this many nanoseconds.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -23,6 +25,11 @@ constexpr int kChunkN = 256;  // centroids per chunk (MMA N)
 constexpr int kBlockK = 64;   // elements of d per K-block (128-byte rows for 16-bit types)
 
 inline long long kpad_of(int K) { return ((long long)K + kChunkN - 1) / kChunkN * kChunkN; }
+
+// Bytes of the tensor-core extension rows of `B` batches: (B, Kpad, 16) 16-bit
+// elements (the norm digits folded into the MMA, fk_norms.cuh).
+constexpr int kExtElems = 16;
+inline size_t ext_bytes(long long B, long long Kpad) { return (size_t)B * Kpad * kExtElems * 2; }
 
 // Counting-sort geometry.
 constexpr int kSortTile = 2048;    // points per sort tile (one warp walks it in order)
@@ -46,7 +53,7 @@ struct Workspace {
   unsigned *maxshift = nullptr;   // device, float bits (non-negative floats order as uints)
   float *h_maxshift = nullptr;    // pinned host mirror
   DevBuf cn, ch, sums, first, counts, offsets, table, digit_off, keys_a, vals_a, keys_b, vals_b;
-  DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2], gsum, gcounts;
+  DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2], gsum, gcounts, xn;
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
 };
@@ -89,18 +96,20 @@ size_t esize(int dtype);
 int num_sms();
 
 // ---- kernels (launchers return fk_status) ----
-// centroid preparation: cn[b, k] = ||c[b,k]||^2 (fp32), +inf on [K, Kpad).
-int launch_prep_cn(const void *c, int dtype, int B, int K, int d, long long Kpad, float *cn,
-                   cudaStream_t s);
-// init for fk_lloyd: master = float(init), ch = init (16-bit dtypes), cn.
+// Centroid preparation for the tensor-core assign: cnx[b, k, 0..15] = the
+// extension row of centroid k (digits of ||c||^2 / 2, see fk_norms.cuh), zero
+// rows on [K, Kpad).  Only for 16-bit dtypes (cnx is (B, Kpad, 16) in dtype).
+int launch_prep_cn(const void *c, int dtype, int B, int K, int d, long long Kpad, void *cnx,
+                   int *err, cudaStream_t s);
+// init for fk_lloyd: master = float(init), ch = init and cnx (16-bit dtypes).
 int launch_init_centers(const void *init, int dtype, int B, int K, int d, long long Kpad,
-                        float *master, void *ch, float *cn, cudaStream_t s);
-// finalize: new = (segment sum) / count or old; max shift; master, ch, cn.
+                        float *master, void *ch, void *cnx, int *err, cudaStream_t s);
+// finalize: new = (segment sum) / count or old; max shift; master, ch, cnx.
 // from_pieces: the segment sum is sums[k] plus the continuation partials of
 // the following pieces (fk_reduce.cu); otherwise sums[k] is complete.
 int launch_finalize(const float *sums, const float *first, int pieces, const int32_t *counts,
-                    const int32_t *offsets, float *centers, void *ch, float *cn, int dtype, int B,
-                    int K, int d, long long Kpad, unsigned *maxshift, bool from_pieces,
+                    const int32_t *offsets, float *centers, void *ch, void *cnx, int dtype, int B,
+                    int K, int d, long long Kpad, unsigned *maxshift, bool from_pieces, int *err,
                     cudaStream_t s);
 // streamed path: gsum[k] += segment sum of one chunk, gcounts[k] += counts[k].
 int launch_accumulate(const float *sums, const float *first, int pieces, const int32_t *counts,
@@ -109,8 +118,14 @@ int launch_accumulate(const float *sums, const float *first, int pieces, const i
 
 int launch_assign_f32(const float *x, const float *c, int B, long long N, int K, int d,
                       int32_t *ids, cudaStream_t s);
-int launch_assign_tc(const void *x, const void *ch, const float *cn, int dtype, int B, long long N,
-                     int K, int d, long long Kpad, int32_t *ids, int *err, cudaStream_t s);
+// cnx: extension rows (B, Kpad, 16) in dtype from launch_prep_cn / finalize;
+// xn: ||x||^2 per point (B, N) from launch_point_norms, or NULL (the kernel
+// then computes it from its shared copy of each point tile).
+int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float *xn, int dtype,
+                     int B, long long N, int K, int d, long long Kpad, int32_t *ids, int *err,
+                     cudaStream_t s);
+// xn[r] = ||x_r||^2 (fp32 accumulation) for `rows` rows of d 16-bit elements.
+int launch_point_norms(const void *x, int dtype, long long rows, int d, float *xn, cudaStream_t s);
 
 // counting sort: counts / offsets optional (workspace offsets are used when
 // NULL); perm always written, keys_out (sorted ids) when not NULL.

@@ -4,15 +4,15 @@
 // assignment: code running under a custom or pooled allocator that owns all
 // device memory, real-time loops that forbid allocation (and the implicit
 // device synchronization that cudaFree can bring), or hosts that only hand
-// out pre-registered buffers.  fk_assign keeps its scratch (the ||c||^2
-// vector and the kernel error word) in a per-stream workspace that it grows
+// out pre-registered buffers.  fk_assign keeps its scratch (the centroid
+// norm rows the tensor-core assign reads and the kernel error word) in a per-stream workspace that it grows
 // with cudaMalloc; this variant instead uses one file-scope static device
 // array, so a call allocates nothing.  The caller still passes the inputs and
 // the output.
 //
 // The array lives on every GPU that loads the library until the process
 // exits.  Its size caps B * Kpad (Kpad = K rounded up to 256) at
-// kNoAllocMaxCn floats.  Host code cannot use the array's name as a device
+// kNoAllocMaxRows norm rows of 32 bytes each.  Host code cannot use the array's name as a device
 // address; the address is looked up once per device with
 // cudaGetSymbolAddress while that device is current.
 #include <mutex>
@@ -22,11 +22,12 @@
 namespace fk {
 namespace {
 
-constexpr long long kNoAllocMaxCn = 1LL << 20;  // floats of ||c||^2 (4 MiB)
-constexpr int kNoAllocHeader = 64;              // floats reserved for the error word
+constexpr long long kNoAllocMaxRows = 1LL << 17;  // norm rows of 16 halves (4 MiB)
+constexpr int kNoAllocHeader = 64;                // floats reserved for the error word
 
-// [0, kNoAllocHeader): error word (int) and padding; then B * Kpad floats of cn.
-static __device__ __align__(256) float g_noalloc_scratch[kNoAllocHeader + kNoAllocMaxCn];
+// [0, kNoAllocHeader): error word (int) and padding; then B * Kpad norm rows.
+static __device__ __align__(256) float
+    g_noalloc_scratch[kNoAllocHeader + kNoAllocMaxRows * kExtElems / 2];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_na_mu;
@@ -68,13 +69,13 @@ extern "C" int fk_assign_noalloc(const void *x, const void *c, int B, long long 
     return set_error(FK_EINVAL, "x and c must be 16-byte aligned");
   if (!tc) return launch_assign_f32((const float *)x, (const float *)c, B, N, K, d, ids, s);
   const long long Kpad = kpad_of(K);
-  if ((long long)B * Kpad > kNoAllocMaxCn)
-    return set_error(FK_EUNSUPPORTED, "fk_assign_noalloc: B * ceil(K/256)*256 exceeds 1048576");
+  if ((long long)B * Kpad > kNoAllocMaxRows)
+    return set_error(FK_EUNSUPPORTED, "fk_assign_noalloc: B * ceil(K/256)*256 exceeds 131072");
   float *base = nullptr;
   FK_TRY(noalloc_base(&base));
   int *err = reinterpret_cast<int *>(base);
-  float *cn = base + kNoAllocHeader;
+  void *cnx = base + kNoAllocHeader;
   FK_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));  // start each call with a clear error word
-  FK_TRY(launch_prep_cn(c, dtype, B, K, d, Kpad, cn, s));
-  return launch_assign_tc(x, c, cn, dtype, B, N, K, d, Kpad, ids, err, s);
+  FK_TRY(launch_prep_cn(c, dtype, B, K, d, Kpad, cnx, err, s));
+  return launch_assign_tc(x, c, cnx, nullptr, dtype, B, N, K, d, Kpad, ids, err, s);
 }

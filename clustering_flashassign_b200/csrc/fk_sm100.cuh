@@ -178,6 +178,19 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
   return desc;
 }
 
+// K-major operand with the 32-byte swizzle: rows of 32 bytes (16 elements of a
+// 16-bit type: one MMA K step), 8-row groups 256 bytes apart (SBO), layout
+// type 6 = SWIZZLE_32B.  The tile base must be 256-byte aligned.
+__device__ __forceinline__ uint64_t desc_k_sw32(uint32_t saddr) {
+  uint64_t desc = 0;
+  desc |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  desc |= (uint64_t)1u << 16;            // leading byte offset (unused for this layout)
+  desc |= (uint64_t)(256u >> 4) << 32;   // stride byte offset
+  desc |= (uint64_t)1u << 46;            // version
+  desc |= (uint64_t)6u << 61;            // SWIZZLE_32B
+  return desc;
+}
+
 // Instruction descriptor of kind::f16 with fp32 accumulation, A and B K-major.
 // ab_fmt: 0 = fp16, 1 = bf16 (A and B always share it).
 __host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_fmt, uint32_t M, uint32_t N) {

@@ -172,10 +172,10 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
  * allocator owning all device memory, or in loops where allocation (and the
  * synchronization a cudaFree can bring) is not allowed, cannot let fk_assign
  * grow its workspace; this call allocates nothing.  Its scratch (the
- * ||c||^2 vector and the kernel error word) is one static device array of
- * 4 MiB + 256 bytes that every GPU loading the library holds until the
- * process exits.
- *   Limit: B * Kpad <= 1048576 for fp16 / bf16, Kpad = K rounded up to a
+ * centroid norm rows, 32 bytes per centroid, and the kernel error word) is
+ * one static device array of 4 MiB + 256 bytes that every GPU loading the
+ * library holds until the process exits.
+ *   Limit: B * Kpad <= 131072 for fp16 / bf16, Kpad = K rounded up to a
  *   multiple of 256; larger shapes return FK_EUNSUPPORTED.  fp32 needs no
  *   scratch and has no such limit.
  *   The first call on a device looks up the array's device address

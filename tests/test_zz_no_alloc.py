@@ -62,7 +62,7 @@ def test_noalloc_assign_matches_fk_assign_on_consecutive_calls():
 def test_noalloc_assign_rejects_shapes_beyond_its_scratch():
     import clustering_flashassign_b200 as fk
     d = ctypes.c_void_p(0x1000)
-    # B * Kpad = 5 * 262144 > 2^20 floats of scratch
-    st = fk.lib.fk_assign_noalloc(d, d, 5, 300000, 262144, 128, fk.FK_F16, d, None)
+    # B * Kpad = 5 * 32768 > 2^17 norm rows of scratch
+    st = fk.lib.fk_assign_noalloc(d, d, 5, 300000, 32768, 128, fk.FK_F16, d, None)
     assert st == fk.FK_EUNSUPPORTED
     assert "exceeds" in fk.fk_last_error()
