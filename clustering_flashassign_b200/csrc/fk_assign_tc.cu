@@ -29,11 +29,11 @@
 //   resident X (d <= 128): the point tile stays in shared memory for all K
 //               chunks (double-buffered across tiles); only centroids stream.
 //               acc = -(||x - c||^2 + 2^-10 ||x||^2) / 2 - 2^-14 < 0, so the
-//               epilogue packs the column into the low 7 mantissa bits of acc
-//               (one LOP3 per value) and keeps a three-input float max (half
-//               an instruction per value).  Columns whose acc agree in all
-//               other bits count as tied and the lowest column wins; that
-//               merges values within 2^-16 of each other (relative).
+//               epilogue packs the column into the low byte of acc (one PRMT
+//               per value) and keeps a three-input float max (half an
+//               instruction per value).  Columns whose acc agree in all other
+//               bits count as tied and the lowest column wins; that merges
+//               values within 2^-15 of each other (relative).
 //   split-d     (d > 128): each pipeline stage carries a 64-wide slice of the
 //               point tile and the matching centroid slice; the d loop runs
 //               inside each K chunk (the pages' split-D path, "flash-kmeans
@@ -64,7 +64,7 @@ constexpr uint32_t kAExtBytes = kTileM * kExt * 2;        // 4 KB of point norm 
 constexpr uint32_t kBExtBytes = kChunkN * kExt * 2;       // 8 KB of centroid norm rows
 constexpr int kExtSlots = 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kKeyMask = 0xFFFFFF80u;  // packed keys: 7 column bits
+constexpr uint32_t kKeyMask = 0xFFFFFF00u;  // packed keys: column in the low byte
 
 struct TcArgs {
   int N;
@@ -126,13 +126,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// Packed key of one accumulator value: acc < 0 with its low 7 mantissa bits
-// replaced by the column.  For negative floats a larger key means a smaller
-// |acc|, and among equal upper bits the smaller column.
-__device__ __forceinline__ float pack_key(uint32_t acc_bits, uint32_t col) {
-  return __uint_as_float((acc_bits & kKeyMask) | col);
-}
-
 __device__ __forceinline__ float key_hi(float key) {
   return __uint_as_float(__float_as_uint(key) & kKeyMask);
 }
@@ -163,16 +156,23 @@ template <> __device__ __forceinline__ void sq2_acc<__nv_bfloat16>(uint32_t v, f
       : "r"(v));
 }
 
-// Running argmax over one 32-column TMEM load, packed keys, four max chains.
-__device__ __forceinline__ void scan_packed(const uint32_t (&r)[32], const uint32_t cb, float &m0,
-                                            float &m1, float &m2, float &m3) {
+// Running argmax over one 32-column TMEM load with packed keys: the low byte
+// of each (negative) accumulator is replaced by its column (a byte taken from
+// colb, which holds the bytes 0..127).  For negative floats a larger key means
+// a smaller |acc|, and among equal upper bits the smaller column.  Four
+// independent max chains.
+__device__ __forceinline__ void scan_packed(const uint32_t (&r)[32], const uint32_t cb,
+                                            const uint32_t (&colb)[32], float &m0, float &m1,
+                                            float &m2, float &m3) {
+#define FK_KEY(t) __uint_as_float(__byte_perm(r[j + (t)], colb[(cb + j + (t)) >> 2], 0x3214u + ((cb + j + (t)) & 3u)))
 #pragma unroll
   for (int j = 0; j < 32; j += 8) {
-    m0 = max3f(m0, pack_key(r[j + 0], cb + j + 0), pack_key(r[j + 1], cb + j + 1));
-    m1 = max3f(m1, pack_key(r[j + 2], cb + j + 2), pack_key(r[j + 3], cb + j + 3));
-    m2 = max3f(m2, pack_key(r[j + 4], cb + j + 4), pack_key(r[j + 5], cb + j + 5));
-    m3 = max3f(m3, pack_key(r[j + 6], cb + j + 6), pack_key(r[j + 7], cb + j + 7));
+    m0 = max3f(m0, FK_KEY(0), FK_KEY(1));
+    m1 = max3f(m1, FK_KEY(2), FK_KEY(3));
+    m2 = max3f(m2, FK_KEY(4), FK_KEY(5));
+    m3 = max3f(m3, FK_KEY(6), FK_KEY(7));
   }
+#undef FK_KEY
 }
 
 // Exact running argmax over one 32-column TMEM load: chain t sees columns
@@ -452,6 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = ew >> 2;   // which 128 columns of each chunk
     const int r_in_tile = quad * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16) + half * 128;
+    uint32_t colb[32];  // bytes 0..127, the column codes of the packed keys
+#pragma unroll
+    for (int i = 0; i < 32; ++i) colb[i] = 0x03020100u + 0x04040404u * i;
     uint32_t h = 0, u = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x, ++u) {
@@ -472,14 +475,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(tb + 96, rd);
         if (RESIDENT) {
           float m0 = best, m1 = best, m2 = best, m3 = best;
-          scan_packed(ra, 0, m0, m1, m2, m3);
-          scan_packed(rb, 32, m0, m1, m2, m3);
+          scan_packed(ra, 0, colb, m0, m1, m2, m3);
+          scan_packed(rb, 32, colb, m0, m1, m2, m3);
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(accempty(ab));  // accumulator may be overwritten
-          scan_packed(rc, 64, m0, m1, m2, m3);
-          scan_packed(rd, 96, m0, m1, m2, m3);
+          scan_packed(rc, 64, colb, m0, m1, m2, m3);
+          scan_packed(rd, 96, colb, m0, m1, m2, m3);
           const float m = fmaxf(max3f(m0, m1, m2), m3);
           // a later chunk must beat the running best in the upper bits
           if (key_hi(m) > key_hi(best)) {
