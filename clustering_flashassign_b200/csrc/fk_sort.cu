@@ -9,16 +9,19 @@
 // stable LSD counting sort by digits of at most 12 bits:
 //   - one pass with the id itself as the digit when K <= 4096,
 //   - two passes (low digit, then high digit) for larger K.
-// Each pass has three kernels:
-//   k_tile_hist    one warp per tile of 2048 points counts digits into its
-//                  own shared-memory counters -> H[b][tile][bin],
-//   k_scan         per batch: bin totals, a block scan over bins -> offsets,
-//                  then the exclusive prefix over tiles of every bin, in place,
-//   k_tile_scatter one warp per tile walks its points in order; equal digits
-//                  inside a round of 32 are ranked with a per-bit ballot mask and
-//                  the warp's cursor per bin starts at offsets[bin] + H[tile].
-// Stability: tiles are ordered by the tile prefix, points inside a tile by the
-// in-order rounds and the lane rank inside a round.
+// Each pass has three kernels over tiles of 2048 points (one CTA of 8 warps
+// per tile; warp w owns the tile's points 256w .. 256w+255, 8 rounds of 32):
+//   k_tile_hist    each warp counts its digits into its own shared counters;
+//                  the CTA sums the 8 warps -> H[b][tile][bin],
+//   k_scan_tiles   per (32 bins, batch): the exclusive prefix over tiles of
+//                  every bin, in place, and the bin totals -> counts,
+//   k_tile_scatter block scan of the counts -> bin offsets (written once per
+//                  batch); per-warp counts again, their prefix over the 8
+//                  warps on top of offsets[bin] + H[tile][bin], then every
+//                  warp ranks its rounds in order: equal digits inside a round
+//                  are ranked with a per-bit ballot mask.
+// Stability: tiles are ordered by the tile prefix, warps inside a tile by the
+// warp prefix, points of a warp by the in-order rounds and the lane rank.
 #include "fk_internal.h"
 
 namespace fk {
@@ -26,8 +29,10 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr unsigned kNoDigit = 0xffffffffu;
-constexpr int kTileWarps = 4;            // warps (= tiles) per CTA
-constexpr int kRounds = kSortTile / 32;  // rounds of 32 points per tile
+constexpr int kSortWarps = 8;                          // warps per tile (CTA)
+constexpr int kWarpPoints = kSortTile / kSortWarps;    // 256 points per warp
+constexpr int kRounds = kWarpPoints / 32;              // rounds of 32 points per warp
+constexpr int kSortThreads = kSortWarps * 32;
 
 struct PassCfg {
   int shift;      // digit = (key >> shift) & mask
@@ -41,11 +46,11 @@ struct PassCfg {
 // digit bit (invalid lanes, digit kNoDigit, match nobody).  Cheaper than a
 // general match instruction for digits of at most 12 bits.
 __device__ __forceinline__ unsigned peers_of(unsigned dg, int nbits) {
-  const bool valid = dg != 0xffffffffu;
-  unsigned peers = __ballot_sync(0xffffffffu, valid);
+  const bool valid = dg != kNoDigit;
+  unsigned peers = __ballot_sync(kFull, valid);
   for (int bit = 0; bit < nbits; ++bit) {
     const bool on = (dg >> bit) & 1u;
-    const unsigned bal = __ballot_sync(0xffffffffu, on);
+    const unsigned bal = __ballot_sync(kFull, on);
     peers &= on ? bal : ~bal;
   }
   return valid ? peers : 0u;
@@ -61,70 +66,50 @@ __device__ __forceinline__ unsigned digit_of(int key, bool valid, const PassCfg 
   return ((unsigned)key >> pc.shift) & pc.mask;
 }
 
-// Copies the tile's values (fewer at the end of a batch) into this warp's shared
-// buffer with asynchronous 4-byte copies (no register round trip, all in
-// flight at once), then waits for them.  Positions past n are zero-filled.
-__device__ __forceinline__ void stage_tile(int32_t *dst, const int32_t *src, long long base,
-                                           long long n, int lane) {
-#pragma unroll 8
+// This warp's keys (kRounds per lane, round r = points 32r..32r+31 of the
+// warp's range), their digits and per-round peer masks.
+struct WarpKeys {
+  int key[kRounds];
+  unsigned dg[kRounds];
+  unsigned peers[kRounds];
+};
+
+__device__ __forceinline__ void load_warp_keys(WarpKeys &wk, const int32_t *kb, long long base,
+                                               int N, const PassCfg &pc, int K, int *err,
+                                               int lane) {
+#pragma unroll
   for (int r = 0; r < kRounds; ++r) {
     const long long i = base + r * 32 + lane;
-    const bool in = i < n;
-    const int32_t *p = src + (in ? i : 0);
-    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst + r * 32 + lane));
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(p), "r"(in ? 4 : 0)
-                 : "memory");
+    wk.key[r] = i < N ? __ldg(kb + i) : 0;
   }
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncwarp();
+#pragma unroll
+  for (int r = 0; r < kRounds; ++r) {
+    const long long i = base + r * 32 + lane;
+    wk.dg[r] = digit_of(wk.key[r], i < N, pc, K, err);
+    wk.peers[r] = peers_of(wk.dg[r], pc.nbits);
+  }
 }
 
-// H[b][tile][bin] = number of points of this tile with this digit.
-__global__ void __launch_bounds__(kTileWarps * 32) k_tile_hist(const int32_t *__restrict__ keys,
-                                                                int N, int K, int T, PassCfg pc,
-                                                                uint32_t *__restrict__ H, int *err) {
-  extern __shared__ uint32_t cnt_all[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x * kTileWarps + warp;
-  const int b = blockIdx.y;
-  if (tile >= T) return;
-  const int bins = pc.bins;
-  uint32_t *cnt = cnt_all + warp * (bins + kSortTile);
-  int32_t *sk = reinterpret_cast<int32_t *>(cnt + bins);
-  const int32_t *kb = keys + (size_t)b * N;
-  const long long base = (long long)tile * kSortTile;
-  stage_tile(sk, kb, base, N, lane);
-  for (int e = lane; e < bins; e += 32) cnt[e] = 0;
-  __syncwarp();
+// cnt[dg] += number of this warp's points with digit dg (one leader per round
+// and digit; the warp owns cnt).
+__device__ __forceinline__ void count_warp(uint32_t *cnt, const WarpKeys &wk, int lane) {
+#pragma unroll
   for (int r = 0; r < kRounds; ++r) {
-    const long long i = base + r * 32 + lane;
-    const bool valid = i < N;
-    const int key = sk[r * 32 + lane];
-    const unsigned dg = digit_of(key, valid, pc, K, err);
-    const unsigned peers = peers_of(dg, pc.nbits);
+    const unsigned dg = wk.dg[r], peers = wk.peers[r];
     if (dg != kNoDigit && lane == __ffs(peers) - 1) cnt[dg] += __popc(peers);
     __syncwarp();
   }
-  uint32_t *hb = H + ((size_t)b * T + tile) * bins;
-  for (int e = lane; e < bins; e += 32) hb[e] = cnt[e];
 }
 
-// One CTA per batch over H[b][T][bins]:
-//   offsets[b][bin] = sum of the totals of earlier bins,
-//   counts[b][bin]  = total of the bin (optional; accumulate adds to it),
-//   H[b][t][bin]    = sum over tiles t' < t of the bin (in place).
-__global__ void __launch_bounds__(1024) k_scan(uint32_t *__restrict__ H, int bins, int T,
-                                               int32_t *__restrict__ counts,
-                                               int32_t *__restrict__ offsets, int accumulate) {
-  __shared__ uint32_t wsum[32];
-  const int b = blockIdx.x;
-  uint32_t *hb = H + (size_t)b * T * bins;
-  const int per = (bins + (int)blockDim.x - 1) / (int)blockDim.x;
-  const int lo = min(bins, (int)threadIdx.x * per), hi = min(bins, lo + per);
+// out[bin] = sum of counts[bin'] over bin' < bin, for bins <= kSortThreads * 16
+// (a block-wide exclusive scan; every thread of the CTA calls it).
+__device__ __forceinline__ void block_excl_scan(const int32_t *counts, int bins, uint32_t *out) {
+  __shared__ uint32_t wsum[kSortWarps];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int per = (bins + kSortThreads - 1) / kSortThreads;
+  const int lo = min(bins, t * per), hi = min(bins, lo + per);
   uint32_t local = 0;
-  for (int bin = lo; bin < hi; ++bin)
-    for (int t = 0; t < T; ++t) local += hb[(size_t)t * bins + bin];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int bin = lo; bin < hi; ++bin) local += (uint32_t)counts[bin];
   uint32_t incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -134,74 +119,144 @@ __global__ void __launch_bounds__(1024) k_scan(uint32_t *__restrict__ H, int bin
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t v = lane < (int)(blockDim.x >> 5) ? wsum[lane] : 0;
+    const uint32_t v = lane < kSortWarps ? wsum[lane] : 0;
     uint32_t vi = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t u = __shfl_up_sync(kFull, vi, o);
       if (lane >= o) vi += u;
     }
-    wsum[lane] = vi - v;
+    if (lane < kSortWarps) wsum[lane] = vi - v;
   }
   __syncthreads();
   uint32_t run = wsum[warp] + incl - local;
   for (int bin = lo; bin < hi; ++bin) {
-    if (offsets) offsets[(size_t)b * bins + bin] = (int32_t)run;
-    uint32_t t_run = 0;
-    for (int t = 0; t < T; ++t) {
-      const uint32_t v = hb[(size_t)t * bins + bin];
-      hb[(size_t)t * bins + bin] = t_run;
-      t_run += v;
+    out[bin] = run;
+    run += (uint32_t)counts[bin];
+  }
+  __syncthreads();
+}
+
+// H[b][tile][bin] = number of points of this tile with this digit.
+__global__ void __launch_bounds__(kSortThreads) k_tile_hist(const int32_t *__restrict__ keys, int N,
+                                                            int K, int T, PassCfg pc,
+                                                            uint32_t *__restrict__ H, int *err) {
+  extern __shared__ uint32_t cnt_all[];  // [kSortWarps][bins]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, b = blockIdx.y;
+  const int bins = pc.bins;
+  for (int e = threadIdx.x; e < kSortWarps * bins; e += kSortThreads) cnt_all[e] = 0;
+  WarpKeys wk;
+  load_warp_keys(wk, keys + (size_t)b * N, (long long)tile * kSortTile + warp * kWarpPoints, N, pc,
+                 K, err, lane);
+  __syncthreads();
+  count_warp(cnt_all + warp * bins, wk, lane);
+  __syncthreads();
+  uint32_t *hb = H + ((size_t)b * T + tile) * bins;
+  for (int bin = threadIdx.x; bin < bins; bin += kSortThreads) {
+    uint32_t t = 0;
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) t += cnt_all[w * bins + bin];
+    hb[bin] = t;
+  }
+}
+
+// Grid (ceil(bins / 32), B): lane = bin, warp w = a contiguous range of tiles.
+//   H[b][t][bin] <- sum over tiles t' < t of the bin (in place),
+//   counts[b][bin] = the bin's total.
+__global__ void __launch_bounds__(kSortThreads) k_scan_tiles(uint32_t *__restrict__ H, int bins,
+                                                             int T, int32_t *__restrict__ counts) {
+  __shared__ uint32_t part[kSortWarps][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y, bin = blockIdx.x * 32 + lane;
+  const bool on = bin < bins;
+  const int per = (T + kSortWarps - 1) / kSortWarps;
+  const int t0 = min(T, warp * per), t1 = min(T, t0 + per);
+  uint32_t *hb = H + (size_t)b * T * bins + bin;
+  uint32_t local = 0;
+  if (on)
+    for (int t = t0; t < t1; ++t) local += hb[(size_t)t * bins];
+  part[warp][lane] = local;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t run = 0;
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) {
+      const uint32_t v = part[w][lane];
+      part[w][lane] = run;
+      run += v;
     }
-    if (counts) {
-      int32_t *dst = counts + (size_t)b * bins + bin;
-      *dst = accumulate ? *dst + (int32_t)t_run : (int32_t)t_run;
+    if (on) counts[(size_t)b * bins + bin] = (int32_t)run;
+  }
+  __syncthreads();
+  if (on) {
+    uint32_t run = part[warp][lane];
+    for (int t = t0; t < t1; ++t) {
+      const uint32_t v = hb[(size_t)t * bins];
+      hb[(size_t)t * bins] = run;
+      run += v;
     }
-    run += t_run;
   }
 }
 
 // Stable scatter: vals_out[pos] = vals_in ? vals_in[i] : i and keys_out[pos] = key,
-// pos = offsets[digit] + H[tile][digit] + rank of the point among the tile's
-// earlier points with the same digit.
-__global__ void __launch_bounds__(kTileWarps * 32) k_tile_scatter(
+// pos = offsets[digit] + G[tile][digit] + (earlier warps of the tile with the
+// digit) + rank of the point among the warp's earlier points with the digit.
+// The CTA of tile 0 also writes offsets_out[b] (when not NULL).
+__global__ void __launch_bounds__(kSortThreads) k_tile_scatter(
     const int32_t *__restrict__ keys, const int32_t *__restrict__ vals_in, int N, int K, int T,
-    PassCfg pc, const uint32_t *__restrict__ G, const int32_t *__restrict__ offsets,
-    int32_t *__restrict__ keys_out, int32_t *__restrict__ vals_out, int *err) {
-  extern __shared__ uint32_t cur_all[];
+    PassCfg pc, const uint32_t *__restrict__ G, const int32_t *__restrict__ counts,
+    int32_t *__restrict__ offsets_out, int32_t *__restrict__ keys_out,
+    int32_t *__restrict__ vals_out, int *err) {
+  extern __shared__ uint32_t sm[];  // off[bins], cnt[kSortWarps][bins]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x * kTileWarps + warp;
-  const int b = blockIdx.y;
-  if (tile >= T) return;
+  const int tile = blockIdx.x, b = blockIdx.y;
   const int bins = pc.bins;
-  uint32_t *cur = cur_all + warp * (bins + 2 * kSortTile);
-  int32_t *sk = reinterpret_cast<int32_t *>(cur + bins);
-  int32_t *sv = sk + kSortTile;
-  const int32_t *kb = keys + (size_t)b * N;
+  uint32_t *off = sm;
+  uint32_t *cnt_all = sm + bins;
+  for (int e = threadIdx.x; e < kSortWarps * bins; e += kSortThreads) cnt_all[e] = 0;
+  block_excl_scan(counts + (size_t)b * bins, bins, off);  // ends with __syncthreads
+  if (tile == 0 && offsets_out)
+    for (int bin = threadIdx.x; bin < bins; bin += kSortThreads)
+      offsets_out[(size_t)b * bins + bin] = (int32_t)off[bin];
+  const long long base = (long long)tile * kSortTile + warp * kWarpPoints;
+  WarpKeys wk;
+  load_warp_keys(wk, keys + (size_t)b * N, base, N, pc, K, err, lane);
+  int vals[kRounds];
+  if (vals_in) {
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r) {
+      const long long i = base + r * 32 + lane;
+      vals[r] = i < N ? __ldg(vals_in + (size_t)b * N + i) : 0;
+    }
+  }
+  uint32_t *cnt = cnt_all + warp * bins;
+  count_warp(cnt, wk, lane);
+  __syncthreads();
+  const uint32_t *gb = G + ((size_t)b * T + tile) * bins;
+  for (int bin = threadIdx.x; bin < bins; bin += kSortThreads) {
+    uint32_t run = off[bin] + gb[bin];
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) {
+      const uint32_t v = cnt_all[w * bins + bin];
+      cnt_all[w * bins + bin] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
   int32_t *ko = keys_out ? keys_out + (size_t)b * N : nullptr;
   int32_t *vo = vals_out + (size_t)b * N;
-  const int32_t *vi = vals_in ? vals_in + (size_t)b * N : nullptr;
-  const long long base = (long long)tile * kSortTile;
-  stage_tile(sk, kb, base, N, lane);
-  if (vi) stage_tile(sv, vi, base, N, lane);
-  const uint32_t *gb = G + ((size_t)b * T + tile) * bins;
-  const int32_t *ob = offsets + (size_t)b * bins;
-  for (int e = lane; e < bins; e += 32) cur[e] = gb[e] + (uint32_t)ob[e];
-  __syncwarp();
   const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
   for (int r = 0; r < kRounds; ++r) {
-    const long long i = base + r * 32 + lane;
-    const bool valid = i < N;
-    const int key = sk[r * 32 + lane];
-    const unsigned dg = digit_of(key, valid, pc, K, err);
-    const unsigned peers = peers_of(dg, pc.nbits);
+    const unsigned dg = wk.dg[r], peers = wk.peers[r];
     uint32_t pos = 0;
-    if (dg != kNoDigit) pos = cur[dg] + __popc(peers & lt);
+    if (dg != kNoDigit) pos = cnt[dg] + __popc(peers & lt);
     __syncwarp();
     if (dg != kNoDigit) {
-      if (lane == __ffs(peers) - 1) cur[dg] += __popc(peers);
-      vo[pos] = vi ? sv[r * 32 + lane] : (int32_t)i;
-      if (ko) ko[pos] = key;
+      if (lane == __ffs(peers) - 1) cnt[dg] += __popc(peers);
+      vo[pos] = vals_in ? vals[r] : (int32_t)(base + r * 32 + lane);
+      if (ko) ko[pos] = wk.key[r];
     }
     __syncwarp();
   }
@@ -231,6 +286,43 @@ __global__ void __launch_bounds__(256) k_count(const int32_t *__restrict__ keys,
   }
 }
 
+// offsets[b][k] = sum of counts[b][k'] over k' < k, one CTA per batch, any K.
+__global__ void __launch_bounds__(1024) k_offsets(const int32_t *__restrict__ counts, int K,
+                                                  int32_t *__restrict__ offsets) {
+  __shared__ uint32_t wsum[32];
+  const int b = blockIdx.x;
+  const int32_t *cb = counts + (size_t)b * K;
+  const int per = (K + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int lo = min(K, (int)threadIdx.x * per), hi = min(K, lo + per);
+  uint32_t local = 0;
+  for (int k = lo; k < hi; ++k) local += (uint32_t)cb[k];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t v = lane < (int)(blockDim.x >> 5) ? wsum[lane] : 0;
+    uint32_t vi = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_up_sync(kFull, vi, o);
+      if (lane >= o) vi += u;
+    }
+    wsum[lane] = vi - v;
+  }
+  __syncthreads();
+  uint32_t run = wsum[warp] + incl - local;
+  for (int k = lo; k < hi; ++k) {
+    offsets[(size_t)b * K + k] = (int32_t)run;
+    run += (uint32_t)cb[k];
+  }
+}
+
 int bits_for(int K) {
   int n = 0;
   while (n < 31 && (1LL << n) < (long long)K) ++n;
@@ -240,8 +332,8 @@ int bits_for(int K) {
 int set_attrs() {
   static bool done = false;
   if (done) return FK_OK;
-  const int hist_max = kTileWarps * ((1 << kMaxDigitBits) + kSortTile) * 4;
-  const int scat_max = kTileWarps * ((1 << kMaxDigitBits) + 2 * kSortTile) * 4;
+  const int hist_max = kSortWarps * (1 << kMaxDigitBits) * 4;
+  const int scat_max = (kSortWarps + 1) * (1 << kMaxDigitBits) * 4;
   FK_CUDA(cudaFuncSetAttribute(k_tile_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, hist_max));
   FK_CUDA(cudaFuncSetAttribute(k_tile_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, scat_max));
   FK_CUDA(cudaFuncSetAttribute(k_count, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
@@ -249,22 +341,25 @@ int set_attrs() {
   return FK_OK;
 }
 
+// One counting-sort pass.  digit_counts (B, bins) receives the digit totals;
+// offsets_out (B, bins), when not NULL, their exclusive scan.
 int one_pass(Workspace *ws, const int32_t *keys_in, const int32_t *vals_in, int B, int N, int K,
-             int T, PassCfg pc, int32_t *counts, int32_t *offsets, bool accumulate,
-             int32_t *keys_out, int32_t *vals_out, cudaStream_t s) {
+             int T, PassCfg pc, int32_t *digit_counts, int32_t *offsets_out, int32_t *keys_out,
+             int32_t *vals_out, cudaStream_t s) {
   FK_TRY(ensure(ws->table, (size_t)B * T * pc.bins * sizeof(uint32_t)));
   uint32_t *H = (uint32_t *)ws->table.p;
-  dim3 grid((unsigned)((T + kTileWarps - 1) / kTileWarps), (unsigned)B);
-  const size_t shm_h = (size_t)kTileWarps * (pc.bins + kSortTile) * sizeof(uint32_t);
-  const size_t shm_s = (size_t)kTileWarps * (pc.bins + 2 * kSortTile) * sizeof(uint32_t);
-  k_tile_hist<<<grid, kTileWarps * 32, shm_h, s>>>(keys_in, N, K, T, pc, H, ws->err);
+  const dim3 grid((unsigned)T, (unsigned)B);
+  const size_t shm_h = (size_t)kSortWarps * pc.bins * sizeof(uint32_t);
+  const size_t shm_s = (size_t)(kSortWarps + 1) * pc.bins * sizeof(uint32_t);
+  k_tile_hist<<<grid, kSortThreads, shm_h, s>>>(keys_in, N, K, T, pc, H, ws->err);
   count_launch();
   FK_CUDA(cudaGetLastError());
-  k_scan<<<B, 1024, 0, s>>>(H, pc.bins, T, counts, offsets, accumulate ? 1 : 0);
+  k_scan_tiles<<<dim3((unsigned)((pc.bins + 31) / 32), (unsigned)B), kSortThreads, 0, s>>>(
+      H, pc.bins, T, digit_counts);
   count_launch();
   FK_CUDA(cudaGetLastError());
-  k_tile_scatter<<<grid, kTileWarps * 32, shm_s, s>>>(keys_in, vals_in, N, K, T, pc, H, offsets,
-                                                    keys_out, vals_out, ws->err);
+  k_tile_scatter<<<grid, kSortThreads, shm_s, s>>>(keys_in, vals_in, N, K, T, pc, H, digit_counts,
+                                                   offsets_out, keys_out, vals_out, ws->err);
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;
@@ -278,6 +373,11 @@ int run_sort(Workspace *ws, const int32_t *ids, int B, long long N_, int K, int3
   const int N = (int)N_;
   const int T = (int)((N_ + kSortTile - 1) / kSortTile);
   const int nbits = bits_for(K);
+  int32_t *cnt = counts;
+  if (!cnt) {
+    FK_TRY(ensure(ws->counts, (size_t)B * K * sizeof(int32_t)));
+    cnt = (int32_t *)ws->counts.p;
+  }
   if (nbits <= kMaxDigitBits) {
     int32_t *off = offsets;
     if (!off) {
@@ -285,41 +385,30 @@ int run_sort(Workspace *ws, const int32_t *ids, int B, long long N_, int K, int3
       off = (int32_t *)ws->offsets.p;
     }
     PassCfg pc{0, 0xffffffffu, K, nbits, true};
-    return one_pass(ws, ids, nullptr, B, N, K, T, pc, counts, off, false, keys_out, perm, s);
+    return one_pass(ws, ids, nullptr, B, N, K, T, pc, cnt, off, keys_out, perm, s);
   }
   const int lo = (nbits + 1) / 2, hi = nbits - lo;
   const size_t nb = (size_t)B * N * sizeof(int32_t);
   FK_TRY(ensure(ws->keys_b, nb));
   FK_TRY(ensure(ws->vals_b, nb));
   int32_t *kt = (int32_t *)ws->keys_b.p, *vt = (int32_t *)ws->vals_b.p;
-  // digit offsets of the passes live in the workspace (at most 4096 per batch)
+  // digit totals of the passes live in the workspace (at most 4096 per batch)
   FK_TRY(ensure(ws->digit_off, (size_t)B * (1 << kMaxDigitBits) * sizeof(int32_t)));
-  int32_t *doff = (int32_t *)ws->digit_off.p;
+  int32_t *dcnt = (int32_t *)ws->digit_off.p;
   PassCfg p1{0, (1u << lo) - 1u, 1 << lo, lo, true};
-  FK_TRY(one_pass(ws, ids, nullptr, B, N, K, T, p1, nullptr, doff, false, kt, vt, s));
+  FK_TRY(one_pass(ws, ids, nullptr, B, N, K, T, p1, dcnt, nullptr, kt, vt, s));
   PassCfg p2{lo, (1u << hi) - 1u, 1 << hi, hi, false};
-  FK_TRY(one_pass(ws, kt, vt, B, N, K, T, p2, nullptr, doff, false, keys_out, perm, s));
-  if (counts || offsets) {
-    int32_t *cnt = counts;
-    if (!cnt) {
-      FK_TRY(ensure(ws->counts, (size_t)B * K * sizeof(int32_t)));
-      cnt = (int32_t *)ws->counts.p;
-    }
-    FK_CUDA(cudaMemsetAsync(cnt, 0, (size_t)B * K * sizeof(int32_t), s));
-    const int use_smem = (size_t)K * 4 <= 64 * 1024 ? 1 : 0;
-    dim3 grid((unsigned)T, (unsigned)B);
-    k_count<<<grid, 256, use_smem ? K * 4 : 0, s>>>(ids, N, K, cnt, use_smem);
+  FK_TRY(one_pass(ws, kt, vt, B, N, K, T, p2, dcnt, nullptr, keys_out, perm, s));
+  // cluster counts and offsets (a pass's digit totals are not cluster totals)
+  FK_CUDA(cudaMemsetAsync(cnt, 0, (size_t)B * K * sizeof(int32_t), s));
+  const int use_smem = (size_t)K * 4 <= 64 * 1024 ? 1 : 0;
+  k_count<<<dim3((unsigned)T, (unsigned)B), 256, use_smem ? K * 4 : 0, s>>>(ids, N, K, cnt, use_smem);
+  count_launch();
+  FK_CUDA(cudaGetLastError());
+  if (offsets) {
+    k_offsets<<<B, 1024, 0, s>>>(cnt, K, offsets);
     count_launch();
     FK_CUDA(cudaGetLastError());
-    if (offsets) {
-      // offsets = exclusive scan of the counts (a table with one tile)
-      FK_TRY(ensure(ws->table, (size_t)B * K * sizeof(uint32_t)));
-      FK_CUDA(cudaMemcpyAsync(ws->table.p, cnt, (size_t)B * K * sizeof(int32_t),
-                              cudaMemcpyDeviceToDevice, s));
-      k_scan<<<B, 1024, 0, s>>>((uint32_t *)ws->table.p, K, 1, nullptr, offsets, 0);
-      count_launch();
-      FK_CUDA(cudaGetLastError());
-    }
   }
   return FK_OK;
 }
