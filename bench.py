@@ -82,29 +82,65 @@ def recorded_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and throttle-reason samples (NVML, every 20 ms) during the timed
+    region; the nvidia-smi query loop is the fallback when NVML is missing."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, period_s=0.02):
         self.idx = gpu_index
+        self.period = period_s
+        self.rows = []
+        self.nvml = None
+        self.thread = None
+        self.stop = False
         self.proc = None
         self.path = None
 
+    def _loop(self, h):
+        import pynvml
+        while not self.stop:
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append((float(sm), float(mx), int(rs)))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
     def __enter__(self):
+        try:
+            import threading
+
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+            self.nvml = pynvml
+            self.thread = threading.Thread(target=self._loop, args=(h,), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.nvml = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
         return self
 
     def __exit__(self, *a):
+        if self.thread is not None:
+            self.stop = True
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -112,38 +148,63 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
-        if not self.path or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+    def _smi_rows(self):
         rows = []
+        if not self.path or not os.path.exists(self.path):
+            return rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                rows.append((float(parts[1]), float(parts[2]), parts))
+                bits = 0
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        bits |= self.BITS[n]
+                rows.append((float(parts[1]), float(parts[2]), bits))
             except ValueError:
                 continue
         os.unlink(self.path)
+        return rows
+
+    def summary(self):
+        rows = self.rows if self.nvml is not None else self._smi_rows()
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         loaded = [r for r in rows if r[0] > 0.5 * r[1]] or rows
-        reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            for n, v in zip(names, r[2][5:9]):
-                if v.strip().lower() == "active":
-                    reasons.add(n)
+        reasons = sorted({n for r in rows for n, bit in self.BITS.items() if r[2] & bit})
         return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": sorted(reasons), "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows),
+                "source": "nvml" if self.nvml is not None else "nvidia-smi"}
+
+
+def rank_workload(rank, **overrides):
+    """The workload of one rank: the same shape on every rank, its own seeds
+    (weak scaling over independent problems: ranks share no data)."""
+    import synthdata
+    w = synthdata.WORKLOADS[WORKLOAD]
+    return synthdata.scaled(w, seed=w.seed + 7919 * rank, init_seed=w.init_seed + 100 * rank, **overrides)
 
 
 def make_inputs(rank):
     import synthdata
-    w = synthdata.WORKLOADS[WORKLOAD]
-    w = synthdata.scaled(w, seed=w.seed + 7919 * rank, init_seed=w.init_seed + 100 * rank)
+    w = rank_workload(rank)
     x, idx, init = synthdata.make(w)
     return w, x, init
+
+
+def reduce_over_ranks(dist, device, to_max, to_sum):
+    """(element-wise max of to_max, element-wise sum of to_sum) over all ranks;
+    the identity without a process group.  Every rank must call it."""
+    if dist is None:
+        return [float(v) for v in to_max], [float(v) for v in to_sum]
+    import torch
+    tmax = torch.tensor([float(v) for v in to_max], dtype=torch.float64, device=device)
+    tsum = torch.tensor([float(v) for v in to_sum], dtype=torch.float64, device=device)
+    dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
+    return [float(v) for v in tmax.tolist()], [float(v) for v in tsum.tolist()]
 
 
 def cpu_oracle_sample(x, init, w, batches, threads=0):
@@ -231,16 +292,7 @@ def run_fk(args, rank, world, local_rank, dist):
     ms = start.elapsed_time(stop)
     clocks = clk.summary()
 
-    if dist is not None:
-        t = torch.tensor([ms, float(iters_total)], device=dev, dtype=torch.float64)
-        tmax = t.clone()
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-        tsum = t.clone()
-        dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
-        ms_max = float(tmax[0])
-        iters_all = float(tsum[1])
-    else:
-        ms_max, iters_all = ms, float(iters_total)
+    (ms_max,), (iters_all,) = reduce_over_ranks(dist, dev, [ms], [iters_total])
 
     # end to end through the C ABI with pinned host buffers
     xh = torch.from_numpy(x).pin_memory()
@@ -264,13 +316,7 @@ def run_fk(args, rank, world, local_rank, dist):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e_ms, float(e_iters)], device=dev, dtype=torch.float64)
-        tmax = t.clone()
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-        tsum = t.clone()
-        dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
-        e_ms, e_iters = float(tmax[0]), float(tsum[1])
+    (e_ms,), (e_iters,) = reduce_over_ranks(dist, dev, [e_ms], [e_iters])
     h2d = x.nbytes + init.nbytes
     d2h = w.B * w.N * 4 + w.B * w.K * w.d * 4
 
@@ -364,7 +410,7 @@ def run_kernel_case(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="fk", choices=["fk", "reference"])
     ap.add_argument("--kernel-case", default=None, choices=["assign", "update"],

@@ -128,6 +128,10 @@ __device__ __forceinline__ float seg_sum(const float *sums, const float *first, 
   return s;
 }
 
+// One warp per centroid (no grid-stride loop, so every centroid's loads are
+// in flight at once).  With d % 4 == 0 lane l handles elements 4l..4l+3,
+// 4l+128.. with 16-byte loads and stores; the arithmetic order per element is
+// the same as in the scalar form.
 template <typename T, bool V4, bool FROM_PIECES>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     k_finalize(const float *__restrict__ sums, const float *__restrict__ first, int pieces,
@@ -136,40 +140,80 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                int d, long long Kpad, unsigned *__restrict__ maxshift, int *err) {
   __shared__ float wmax[kWarpsPerBlock];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long w = (long long)blockIdx.x * kWarpsPerBlock + warp;
   float my_max = 0.f;
-  for (long long w = (long long)blockIdx.x * kWarpsPerBlock + warp; w < (long long)B * K;
-       w += (long long)gridDim.x * kWarpsPerBlock) {
+  if (w < (long long)B * K) {
     const int b = (int)(w / K), k = (int)(w % K);
-    const int cnt = counts[w];
+    const int cnt = __ldg(counts + w);
     int p0 = 0, pl = -1;
     if (FROM_PIECES && cnt > 0) {
-      const int off = offsets[w];
+      const int off = __ldg(offsets + w);
       p0 = off / kPiece;
       pl = (off + cnt - 1) / kPiece;
     }
     const size_t w_off = (size_t)w * d;
     const size_t first_b = (size_t)b * pieces * d;
     float shift2 = 0.f, nrm = 0.f;
-    for_lane_elems<V4>(d, lane, [&](int j, int n) {
-      for (int e = 0; e < n; ++e) {
-        const float old = centers[w_off + j + e];
-        float nv = old;
-        if (cnt > 0) nv = seg_sum<FROM_PIECES>(sums, first, w_off, first_b, d, p0, pl, j + e) / (float)cnt;
-        const float t = nv - old;
-        shift2 = fmaf(t, t, shift2);
-        centers[w_off + j + e] = nv;
+    if (V4) {
+      for (int j = lane * 4; j < d; j += 128) {
+        const float4 old = *reinterpret_cast<const float4 *>(centers + w_off + j);
+        float4 nv = old;
+        if (cnt > 0) {
+          float4 sm = __ldg(reinterpret_cast<const float4 *>(sums + w_off + j));
+          if (FROM_PIECES)
+            for (int p = p0 + 1; p <= pl; ++p) {
+              const float4 f = __ldg(reinterpret_cast<const float4 *>(first + first_b + (size_t)p * d + j));
+              sm.x += f.x;
+              sm.y += f.y;
+              sm.z += f.z;
+              sm.w += f.w;
+            }
+          nv = make_float4(sm.x / (float)cnt, sm.y / (float)cnt, sm.z / (float)cnt, sm.w / (float)cnt);
+        }
+        const float o4[4] = {old.x, old.y, old.z, old.w};
+        const float n4[4] = {nv.x, nv.y, nv.z, nv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float t = n4[e] - o4[e];
+          shift2 = fmaf(t, t, shift2);
+        }
+        *reinterpret_cast<float4 *>(centers + w_off + j) = nv;
         if (ch) {
-          const T r = from_f<T>(nv);
-          ch[w_off + j + e] = r;
-          const float rf = to_f<T>(r);
-          nrm = fmaf(rf, rf, nrm);
+          alignas(8) T r4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            r4[e] = from_f<T>(n4[e]);
+            const float rf = to_f<T>(r4[e]);
+            nrm = fmaf(rf, rf, nrm);
+          }
+          if constexpr (sizeof(T) == 2)
+            *reinterpret_cast<uint2 *>(ch + w_off + j) = *reinterpret_cast<const uint2 *>(r4);
+          else
+            for (int e = 0; e < 4; ++e) ch[w_off + j + e] = r4[e];
         }
       }
-    });
+    } else {
+      for_lane_elems<V4>(d, lane, [&](int j, int n) {
+        for (int e = 0; e < n; ++e) {
+          const float old = centers[w_off + j + e];
+          float nv = old;
+          if (cnt > 0) nv = seg_sum<FROM_PIECES>(sums, first, w_off, first_b, d, p0, pl, j + e) / (float)cnt;
+          const float t = nv - old;
+          shift2 = fmaf(t, t, shift2);
+          centers[w_off + j + e] = nv;
+          if (ch) {
+            const T r = from_f<T>(nv);
+            ch[w_off + j + e] = r;
+            const float rf = to_f<T>(r);
+            nrm = fmaf(rf, rf, nrm);
+          }
+        }
+      });
+    }
     shift2 = warp_sum(shift2);
     nrm = warp_sum(nrm);
     if (lane == 0 && cnx) store_ext<T>(cnx, (long long)b * Kpad + k, true, nrm, err);
-    my_max = fmaxf(my_max, sqrtf(shift2));
+    my_max = sqrtf(shift2);
   }
   if (lane == 0) wmax[warp] = my_max;
   __syncthreads();
@@ -235,9 +279,7 @@ template <typename T, bool FP>
 int fin_t(const float *sums, const float *first, int pieces, const int32_t *counts,
           const int32_t *offsets, float *centers, void *ch, void *cnx, int B, int K, int d,
           long long Kpad, unsigned *maxshift, int *err, cudaStream_t s) {
-  unsigned g = blocks_for((long long)B * K);
-  const unsigned cap = (unsigned)num_sms() * 8;
-  if (g > cap) g = cap;
+  const unsigned g = blocks_for((long long)B * K);
   if (d % 4 == 0)
     k_finalize<T, true, FP><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, centers,
                                                               (T *)ch, (T *)cnx, B, K, d, Kpad, maxshift, err);
