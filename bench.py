@@ -379,6 +379,99 @@ def run_fk(args, rank, world, local_rank, dist):
     print(json.dumps(line), flush=True)
 
 
+def run_largen(args):
+    """The large-N streamed workload (B=1, N=2^28, K=32768, d=128, fp16 mixture,
+    64 GiB of points in pinned host memory), 3 Lloyd iterations per step.  The
+    points are re-streamed every iteration in 2^24-point chunks whose copies
+    overlap the compute.  Reports iterations/s, the effective and the measured
+    peak pinned host-to-device bandwidth, and the ideal iteration time
+    max(tensor time, copy time) against the measured one."""
+    import numpy as np
+    import torch
+
+    import clustering_flashassign_b200 as fk
+    import oracle
+    import synthdata
+    w = synthdata.WORKLOADS["largen"]
+    if args.points:
+        w = synthdata.scaled(w, N=args.points)
+    t0 = time.perf_counter()
+    xt = torch.empty((w.B, w.N, w.d), dtype=torch.float16, pin_memory=True)
+    _, _, init = synthdata.make(w, out=xt.numpy())
+    gen_s = time.perf_counter() - t0
+    dev = torch.device("cuda", 0)
+    initd = torch.from_numpy(init).to(dev)
+    ids = torch.empty((w.B, w.N), dtype=torch.int32, device=dev)
+    cen = torch.empty((w.B, w.K, w.d), dtype=torch.float32, device=dev)
+
+    # pinned host -> device copy peak (one 2^24-point chunk, best of 3)
+    chunk = min(w.N, 1 << 24)
+    dst = torch.empty((chunk, w.d), dtype=torch.float16, device=dev)
+    src = xt[0, :chunk]
+    best = 1e30
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dst.copy_(src, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    h2d_peak = chunk * w.d * 2 / (best * 1e-3) / 1e9
+    del dst
+
+    fk.fk_lloyd(xt, initd, 1, 0.0, ids, cen, host_mode=fk.FK_HOST_STREAM)  # warm-up (workspace)
+    torch.cuda.synchronize()
+    fk.fk_profile_read(reset=True)
+    fk.fk_profile_enable(True)
+    launches0 = fk.fk_launch_count()
+    iters = 0
+    with ClockSampler(0) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            iters += fk.fk_lloyd(xt, initd, w.iters, 0.0, ids, cen, host_mode=fk.FK_HOST_STREAM)
+        e1.record()
+        torch.cuda.synchronize()
+    fk.fk_profile_enable(False)
+    prof = fk.fk_profile_read(reset=True)
+    ms = e0.elapsed_time(e1)
+    peaks, src_name = load_peaks()
+    peak_t = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    flop_iter = 2.0 * w.B * w.N * w.K * w.d
+    bytes_iter = w.B * w.N * w.d * 2
+    iter_ms = ms / iters
+    ideal_ms = max(flop_iter / (peak_t * 1e12), bytes_iter / (h2d_peak * 1e9)) * 1e3
+    a_ms = prof["assign_ms"] / iters
+    # checker: one iteration on the first 2^14 points with all K, extrapolated
+    ns = 1 << 14
+    xs = np.ascontiguousarray(xt.numpy()[:, :ns])
+    c0 = synthdata.to_f64(init, w.dtype)
+    tc = time.perf_counter()
+    cid, _, _ = oracle.assign(xs, w.dtype, c0)
+    oracle.update(xs, w.dtype, cid, c0)
+    cpu_iter_s = (time.perf_counter() - tc) * (w.N / ns)
+    line = {
+        "metric": "Lloyd iter/s, large-N streamed from pinned host memory",
+        "value": iters / (ms * 1e-3), "unit": "iter/s", "n_gpus": 1, "steps": args.steps, "warmup": 1,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": f"largen: B={w.B} N={w.N} K={w.K} d={w.d} {w.dtype} mixture, points in pinned "
+                               f"host memory, 2^24-point chunks, {w.iters} iterations per step",
+                   "host_bytes": bytes_iter, "generation_s": gen_s},
+        "roofline": {"bound": "max(tensor, pcie)", "achieved_ms_per_iter": iter_ms, "ideal_ms_per_iter": ideal_ms,
+                     "frac": ideal_ms / iter_ms, "h2d_peak_gbs": h2d_peak,
+                     "h2d_effective_gbs": bytes_iter / (iter_ms * 1e-3) / 1e9,
+                     "assign_tflops": flop_iter / (a_ms * 1e-3) / 1e12 if a_ms > 0 else None,
+                     "tensor_peak_tflops": peak_t, "peak_source": src_name},
+        "cpu_baseline": {"value": 1.0 / cpu_iter_s, "unit": "iter/s", "cores": oracle.max_threads(),
+                         "kind": "oracle",
+                         "sample": f"one iteration on the first {ns} points with all K, extrapolated x{w.N // ns}"},
+        "gpu_launches": fk.fk_launch_count() - launches0,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_kernel_case(args):
     """Launch only one step kind on the bench workload (for profiler captures):
     assign = fk_assign, update = fk_update, each warmup + steps times."""
@@ -415,7 +508,9 @@ def main():
     ap.add_argument("--impl", default="fk", choices=["fk", "reference"])
     ap.add_argument("--kernel-case", default=None, choices=["assign", "update"],
                     help="launch only this step (profiler captures); prints no bench line")
-    ap.add_argument("--points", type=int, default=0, help="with --kernel-case: points per batch")
+    ap.add_argument("--points", type=int, default=0, help="with --kernel-case / --workload: points per batch")
+    ap.add_argument("--workload", default="api", choices=["api", "largen"],
+                    help="largen: the 64 GiB streamed workload (its own line; not the default bench)")
     args = ap.parse_args()
     world = env_int("WORLD_SIZE", 1)
     rank = env_int("RANK", 0)
@@ -425,6 +520,9 @@ def main():
         return
     if args.kernel_case:
         run_kernel_case(args)
+        return
+    if args.workload == "largen":
+        run_largen(args)
         return
     dist = None
     if world > 1:
