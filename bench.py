@@ -179,17 +179,23 @@ class ClockSampler:
                 "source": "nvml" if self.nvml is not None else "nvidia-smi"}
 
 
-def rank_workload(rank, **overrides):
+def metric_for(w):
+    if w.name == WORKLOAD:
+        return METRIC
+    return f"Lloyd iter/s at B{w.B}·N{w.N}·K{w.K}·d{w.d} {w.dtype}; assign TFLOP/s; update GB/s"
+
+
+def rank_workload(rank, name=WORKLOAD, **overrides):
     """The workload of one rank: the same shape on every rank, its own seeds
     (weak scaling over independent problems: ranks share no data)."""
     import synthdata
-    w = synthdata.WORKLOADS[WORKLOAD]
+    w = synthdata.WORKLOADS[name]
     return synthdata.scaled(w, seed=w.seed + 7919 * rank, init_seed=w.init_seed + 100 * rank, **overrides)
 
 
-def make_inputs(rank):
+def make_inputs(rank, name=WORKLOAD):
     import synthdata
-    w = rank_workload(rank)
+    w = rank_workload(rank, name)
     x, idx, init = synthdata.make(w)
     return w, x, init
 
@@ -254,9 +260,14 @@ def run_fk(args, rank, world, local_rank, dist):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w, x, init = make_inputs(rank)
-    xd = torch.from_numpy(x).to(dev)
-    initd = torch.from_numpy(init).to(dev)
+    w, x, init = make_inputs(rank, args.workload)
+
+    def as_torch(a):  # bf16 arrays are stored as uint16 bit patterns
+        t = torch.from_numpy(a)
+        return t.view(torch.bfloat16) if w.dtype == "bf16" else t
+
+    xd = as_torch(x).to(dev)
+    initd = as_torch(init).to(dev)
     ids = torch.empty((w.B, w.N), dtype=torch.int32, device=dev)
     centers = torch.empty((w.B, w.K, w.d), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -295,8 +306,8 @@ def run_fk(args, rank, world, local_rank, dist):
     (ms_max,), (iters_all,) = reduce_over_ranks(dist, dev, [ms], [iters_total])
 
     # end to end through the C ABI with pinned host buffers
-    xh = torch.from_numpy(x).pin_memory()
-    inith = torch.from_numpy(init).pin_memory()
+    xh = as_torch(x).pin_memory()
+    inith = as_torch(init).pin_memory()
     idsh = torch.empty((w.B, w.N), dtype=torch.int32).pin_memory()
     cenh = torch.empty((w.B, w.K, w.d), dtype=torch.float32).pin_memory()
 
@@ -327,8 +338,17 @@ def run_fk(args, rank, world, local_rank, dist):
     flop = 2.0 * w.B * w.N * w.K * w.d
     a_ms = prof["assign_ms"] / max(1, prof["assign_launches"])
     achieved = flop / (a_ms * 1e-3) / 1e12
-    peak_t = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])  # fp16 rate = bf16 rate
-    traffic = recorded_traffic()
+    if w.dtype == "f32":
+        # fp32 inputs take the SIMT kernel: peak from unit counts and the max clock
+        mhz = float(peaks.get("sm_max_mhz", 1965.0))
+        peak_t = 148 * 128 * 2 * mhz * 1e6 / 1e12
+        bound, kname = "alu", "fp32 SIMT assign (k_assign_f32)"
+        psrc = f"derived: 148 SMs x 128 fp32 lanes x 2 flop x {mhz:.0f} MHz"
+    else:
+        peak_t = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])  # fp16 rate = bf16 rate
+        bound, kname = "tensor", "FlashAssign (k_flash_assign)"
+        psrc = f"{src} bf16 dense, sustained (fp16 runs at the bf16 rate)"
+    traffic = recorded_traffic() if w.name == WORKLOAD else None
     s = 2 if w.dtype != "f32" else 4
     upd_bytes = (w.B * w.N * w.d * s + 8 * w.B * w.N + 8 * w.B * w.N + 16 * w.B * w.K * w.d
                  + 2 * w.B * w.K * w.d + 12 * w.B * w.K)
@@ -337,12 +357,12 @@ def run_fk(args, rank, world, local_rank, dist):
     hbm = float(peaks["hbm_gbs"])
 
     import oracle
-    batches = 4
+    batches = min(4, w.B)
     cpu_t = cpu_oracle_sample(x, init, w, batches)
     cpu_value = 1.0 / (cpu_t * w.B / batches)
 
     line = {
-        "metric": METRIC,
+        "metric": metric_for(w),
         "value": iters_all / (ms_max * 1e-3),
         "unit": "iter/s",
         "n_gpus": world,
@@ -354,15 +374,16 @@ def run_fk(args, rank, world, local_rank, dist):
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD}: B={w.B} N={w.N} K={w.K} d={w.d} {w.dtype} points ~ N(0,1), "
-                               f"{w.iters} iterations max, tol={w.tol}",
+        "config": {"workload": f"{w.name}: B={w.B} N={w.N} K={w.K} d={w.d} {w.dtype} "
+                               + ("points ~ N(0,1), " if w.n_comp <= 1 else f"{w.n_comp}-component mixture, ")
+                               + f"{w.iters} iterations max, tol={w.tol}",
                    "B": w.B, "N": w.N, "K": w.K, "d": w.d, "iterations_per_rank": iters_total,
-                   "l2": "inputs larger than L2 (points 619 MB per rank)",
+                   "l2": (f"inputs larger than L2 (points {x.nbytes / 1e6:.0f} MB per rank)" if x.nbytes > 126e6
+                          else f"points {x.nbytes / 1e6:.0f} MB per rank (fit in L2)"),
                    "parallelism": f"independent problems, {world} rank(s)"},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": achieved / peak_t, "traffic": traffic,
-                     "kernel": "FlashAssign (k_flash_assign)", "ms_per_launch": a_ms,
-                     "peak_source": f"{src} bf16 dense, sustained (fp16 runs at the bf16 rate)"},
+                     "kernel": kname, "ms_per_launch": a_ms, "peak_source": psrc},
         "kernels": {"assign_tflops": achieved, "assign_frac": achieved / peak_t,
                     "update_gbs": upd_gbs, "update_frac_of_hbm": upd_gbs / hbm,
                     "update_ms": upd_ms, "sort_ms": prof["sort_ms"] / max(1, prof["update_calls"]),
@@ -509,8 +530,9 @@ def main():
     ap.add_argument("--kernel-case", default=None, choices=["assign", "update"],
                     help="launch only this step (profiler captures); prints no bench line")
     ap.add_argument("--points", type=int, default=0, help="with --kernel-case / --workload: points per batch")
-    ap.add_argument("--workload", default="api", choices=["api", "largen"],
-                    help="largen: the 64 GiB streamed workload (its own line; not the default bench)")
+    ap.add_argument("--workload", default="api", choices=["api", "tiny", "zipf", "splitd", "largen"],
+                    help="api is the benchmark; the others print their own line (largen: the 64 GiB "
+                         "streamed workload)")
     args = ap.parse_args()
     world = env_int("WORLD_SIZE", 1)
     rank = env_int("RANK", 0)
