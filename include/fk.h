@@ -95,6 +95,12 @@ typedef struct {
  *   x    (B, N, d) in dtype, device.  c (B, K, d) in dtype, device.
  *   ids  (B, N) int32 out, device.
  * fp16 / bf16 run on tcgen05 tensor cores (TMA-fed tiles, TMEM accumulators);
+ * the squared norms enter the accumulator through one extra K = 16 MMA step,
+ * so the ranking value is ||x - c||^2 (+ a per-point constant) in fp32.  For
+ * d <= 128 the argmin keeps the column in the low byte of that fp32 value:
+ * values within 2^-15 of each other (relative) count as tied and the lowest
+ * k wins.  fp16 inputs need ||c||^2 and ||x||^2 below 2^32; beyond that the
+ * device error word records FK_EUNSUPPORTED (fk_device_error()).
  * fp32 runs on CUDA cores and evaluates sum_j (x_j - c_j)^2 directly (same
  * argmin, no cancellation).
  */
@@ -106,7 +112,8 @@ int fk_assign(const void *x, const void *c, int B, long long N, int K, int d, in
  * counts[b,k] = #{i : ids[b,i] = k};  centers[b,k] = mean of its points in
  * fp32, or unchanged when counts[b,k] = 0.  The points are gathered in
  * sorted order without being permuted; each segment piece is reduced on chip
- * and flushed with one vector atomic add.
+ * and stored once (no atomics: a segment spread over several pieces is summed
+ * in piece order by the finalize), so the result is bit-reproducible.
  * Passage: "Flash-KMeans: IO感知的精确K-Means", section "它攻克的兩大瓶頸"
  * (argsort of the assignment vector, contiguous segments, one atomic add per
  * segment); "Flash-KMeans: Fast and Memory-Efficient Exact K-Means",
