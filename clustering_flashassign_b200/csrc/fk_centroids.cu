@@ -33,6 +33,10 @@ template <> __device__ __forceinline__ float from_f<float>(float v) { return v; 
 template <> __device__ __forceinline__ __half from_f<__half>(float v) { return __float2half_rn(v); }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
 
+__device__ __forceinline__ uint16_t bits16(__half v) { return __half_as_ushort(v); }
+__device__ __forceinline__ uint16_t bits16(__nv_bfloat16 v) { return __bfloat16_as_ushort(v); }
+__device__ __forceinline__ uint16_t bits16(float) { return 0; }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -145,9 +149,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   if (w < (long long)B * K) {
     const int b = (int)(w / K), k = (int)(w % K);
     const int cnt = __ldg(counts + w);
+    const int off = FROM_PIECES ? __ldg(offsets + w) : 0;  // both loads in flight together
     int p0 = 0, pl = -1;
     if (FROM_PIECES && cnt > 0) {
-      const int off = __ldg(offsets + w);
       p0 = off / kPiece;
       pl = (off + cnt - 1) / kPiece;
     }
@@ -179,17 +183,25 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         }
         *reinterpret_cast<float4 *>(centers + w_off + j) = nv;
         if (ch) {
-          alignas(8) T r4[4];
+          if constexpr (sizeof(T) == 2) {
+            uint32_t packed[2] = {0u, 0u};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            r4[e] = from_f<T>(n4[e]);
-            const float rf = to_f<T>(r4[e]);
-            nrm = fmaf(rf, rf, nrm);
+            for (int e = 0; e < 4; ++e) {
+              const T r = from_f<T>(n4[e]);
+              const float rf = to_f<T>(r);
+              nrm = fmaf(rf, rf, nrm);
+              packed[e >> 1] |= (uint32_t)bits16(r) << (16 * (e & 1));
+            }
+            *reinterpret_cast<uint2 *>(ch + w_off + j) = make_uint2(packed[0], packed[1]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const T r = from_f<T>(n4[e]);
+              ch[w_off + j + e] = r;
+              const float rf = to_f<T>(r);
+              nrm = fmaf(rf, rf, nrm);
+            }
           }
-          if constexpr (sizeof(T) == 2)
-            *reinterpret_cast<uint2 *>(ch + w_off + j) = *reinterpret_cast<const uint2 *>(r4);
-          else
-            for (int e = 0; e < 4; ++e) ch[w_off + j + e] = r4[e];
         }
       }
     } else {
