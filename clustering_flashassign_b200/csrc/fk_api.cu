@@ -350,17 +350,42 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
     }
     FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cnx, ws->err, s));
     const void *cassign = dtype == FK_F32 ? (const void *)cen_dev : ch;
+    // The assign of iteration it+1 is queued before the host looks at the
+    // shift of iteration it, so the GPU never idles during the tol check.  It
+    // writes the other of two id buffers: when the check stops the loop, the
+    // returned ids are still those of the last assign whose update produced
+    // the returned centroids, and the queued assign is discarded.
+    const bool check = tol > 0.f || o.verbose;
+    int32_t *idbuf[2] = {ids_dev, ids_dev};
+    if (check && max_iter > 1) {
+      FK_TRY(ensure(ws->ids_alt, (size_t)B * N * sizeof(int32_t)));
+      idbuf[1] = (int32_t *)ws->ids_alt.p;
+      if (!ws->shift_ev) FK_CUDA(cudaEventCreateWithFlags(&ws->shift_ev, cudaEventDisableTiming));
+    }
+    int cur = 0;
+    if (max_iter > 0)
+      FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, idbuf[0], s));
     for (int it = 0; it < max_iter; ++it) {
-      FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, ids_dev, s));
-      FK_TRY(do_update(ws, xdev, ids_dev, B, N, K, d, dtype, cen_dev, nullptr, ch, cnx, Kpad, s));
+      FK_TRY(do_update(ws, xdev, idbuf[cur], B, N, K, d, dtype, cen_dev, nullptr, ch, cnx, Kpad, s));
       iters = it + 1;
-      if (tol > 0.f || o.verbose) {
-        float ms = 0.f;
-        FK_TRY(read_shift(ws, s, &ms));
+      const bool last = it + 1 == max_iter;
+      if (check) {
+        FK_CUDA(cudaMemcpyAsync(ws->h_maxshift, ws->maxshift, sizeof(float), cudaMemcpyDeviceToHost, s));
+        if (ws->shift_ev) FK_CUDA(cudaEventRecord(ws->shift_ev, s));
+        if (!last)
+          FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, idbuf[cur ^ 1], s));
+        if (ws->shift_ev) FK_CUDA(cudaEventSynchronize(ws->shift_ev));
+        else FK_CUDA(cudaStreamSynchronize(s));
+        const float ms = *ws->h_maxshift;
         if (o.verbose) fprintf(stderr, "fk_lloyd iter %d max_shift %.6g\n", it + 1, ms);
         if (tol > 0.f && ms < tol) break;
+        if (!last) cur ^= 1;
+      } else if (!last) {
+        FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, idbuf[0], s));
       }
     }
+    if (idbuf[cur] != ids_dev)
+      FK_CUDA(cudaMemcpyAsync(ids_dev, idbuf[cur], (size_t)B * N * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
   }
   if (ids_dev != ids)
     FK_CUDA(cudaMemcpyAsync(ids, ids_dev, (size_t)B * N * sizeof(int32_t), cudaMemcpyDeviceToHost, s));

@@ -53,9 +53,10 @@ struct Workspace {
   unsigned *maxshift = nullptr;   // device, float bits (non-negative floats order as uints)
   float *h_maxshift = nullptr;    // pinned host mirror
   DevBuf cn, ch, sums, first, counts, offsets, table, digit_off, keys_a, vals_a, keys_b, vals_b;
-  DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2], gsum, gcounts, xn;
+  DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2], gsum, gcounts, xn, ids_alt;
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
+  cudaEvent_t shift_ev = nullptr;  // the max-shift copy of the Lloyd loop has landed
 };
 
 // Status plumbing (thread-local last-error text).

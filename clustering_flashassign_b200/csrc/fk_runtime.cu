@@ -108,7 +108,7 @@ int release_device_workspaces() {
     DevBuf *bufs[] = {&ws->cn, &ws->ch, &ws->sums, &ws->first, &ws->counts, &ws->offsets,
                       &ws->table, &ws->digit_off, &ws->keys_a, &ws->vals_a, &ws->keys_b,
                       &ws->vals_b, &ws->xres, &ws->init_dev, &ws->ids_dev, &ws->centers_dev,
-                      &ws->chunk[0], &ws->chunk[1], &ws->gsum, &ws->gcounts, &ws->xn};
+                      &ws->chunk[0], &ws->chunk[1], &ws->gsum, &ws->gcounts, &ws->xn, &ws->ids_alt};
     for (DevBuf *b : bufs) free_buf(*b);
     if (ws->err) cudaFree(ws->err);
     if (ws->h_maxshift) cudaFreeHost(ws->h_maxshift);
@@ -117,6 +117,7 @@ int release_device_workspaces() {
       if (ws->ready[i]) cudaEventDestroy(ws->ready[i]);
       if (ws->freed[i]) cudaEventDestroy(ws->freed[i]);
     }
+    if (ws->shift_ev) cudaEventDestroy(ws->shift_ev);
     delete ws;
     it = g_ws.erase(it);
   }
