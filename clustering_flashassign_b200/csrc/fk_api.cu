@@ -70,9 +70,11 @@ int prepare_update(Workspace *ws, int B, long long n, int K, int d) {
 
 // Steps a2-a5 on device-resident points; ch / cnx (nullable) receive the dtype
 // copy and the tensor-core extension rows of the new centroids for the next assign.
+// have_hist: ws->table already holds the sort's tile histogram (accumulated by
+// the assign), so the sort skips its histogram kernel.
 int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long N, int K, int d,
               int dtype, float *centers, int32_t *counts_out, void *ch, void *cnx, long long Kpad,
-              cudaStream_t s) {
+              cudaStream_t s, bool have_hist = false) {
   note_update_call();
   int32_t *counts = counts_out;
   if (!counts) {
@@ -86,7 +88,8 @@ int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long
   float *sums = (float *)ws->sums.p, *first = (float *)ws->first.p;
   {
     PhaseTimer t(PH_SORT, s);
-    FK_TRY(run_sort(ws, ids, B, N, K, counts, offsets, perm, keys, s));
+    if (have_hist) FK_TRY(run_sort_prehist(ws, ids, B, N, K, counts, offsets, perm, keys, s));
+    else FK_TRY(run_sort(ws, ids, B, N, K, counts, offsets, perm, keys, s));
   }
   {
     PhaseTimer t(PH_REDUCE, s);
@@ -99,10 +102,10 @@ int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long
 
 int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const void *cnx,
                        const float *xn, int B, long long N, int K, int d, int dtype, long long Kpad,
-                       int32_t *ids, cudaStream_t s) {
+                       int32_t *ids, cudaStream_t s, uint32_t *hist = nullptr) {
   PhaseTimer t(PH_ASSIGN, s);
   if (dtype == FK_F32) return launch_assign_f32((const float *)x, (const float *)cdt, B, N, K, d, ids, s);
-  return launch_assign_tc(x, cdt, cnx, xn, dtype, B, N, K, d, Kpad, ids, ws->err, s);
+  return launch_assign_tc(x, cdt, cnx, xn, dtype, B, N, K, d, Kpad, ids, ws->err, s, hist);
 }
 
 int read_shift(Workspace *ws, cudaStream_t s, float *out) {
@@ -362,18 +365,29 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
       idbuf[1] = (int32_t *)ws->ids_alt.p;
       if (!ws->shift_ev) FK_CUDA(cudaEventCreateWithFlags(&ws->shift_ev, cudaEventDisableTiming));
     }
+    // With K <= 4096 the tensor-core assign also counts every id into the
+    // sort's tile histogram, so the sort starts at its scan.
+    const bool fuse = dtype != FK_F32 && sort_single_pass(K);
+    uint32_t *hist = nullptr;
+    const size_t hist_bytes = sort_table_bytes(B, N, K);
+    if (fuse) {
+      FK_TRY(ensure(ws->table, hist_bytes));
+      hist = (uint32_t *)ws->table.p;
+    }
+    auto assign = [&](int32_t *out) -> int {
+      if (hist) FK_CUDA(cudaMemsetAsync(hist, 0, hist_bytes, s));
+      return do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, out, s, hist);
+    };
     int cur = 0;
-    if (max_iter > 0)
-      FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, idbuf[0], s));
+    if (max_iter > 0) FK_TRY(assign(idbuf[0]));
     for (int it = 0; it < max_iter; ++it) {
-      FK_TRY(do_update(ws, xdev, idbuf[cur], B, N, K, d, dtype, cen_dev, nullptr, ch, cnx, Kpad, s));
+      FK_TRY(do_update(ws, xdev, idbuf[cur], B, N, K, d, dtype, cen_dev, nullptr, ch, cnx, Kpad, s, fuse));
       iters = it + 1;
       const bool last = it + 1 == max_iter;
       if (check) {
         FK_CUDA(cudaMemcpyAsync(ws->h_maxshift, ws->maxshift, sizeof(float), cudaMemcpyDeviceToHost, s));
         if (ws->shift_ev) FK_CUDA(cudaEventRecord(ws->shift_ev, s));
-        if (!last)
-          FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, idbuf[cur ^ 1], s));
+        if (!last) FK_TRY(assign(idbuf[cur ^ 1]));
         if (ws->shift_ev) FK_CUDA(cudaEventSynchronize(ws->shift_ev));
         else FK_CUDA(cudaStreamSynchronize(s));
         const float ms = *ws->h_maxshift;
@@ -381,7 +395,7 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
         if (tol > 0.f && ms < tol) break;
         if (!last) cur ^= 1;
       } else if (!last) {
-        FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, idbuf[0], s));
+        FK_TRY(assign(idbuf[0]));
       }
     }
     if (idbuf[cur] != ids_dev)

@@ -68,6 +68,7 @@ constexpr uint32_t kKeyMask = 0xFFFFFF00u;  // packed keys: column in the low by
 
 struct TcArgs {
   int N;
+  int K;
   int tiles_per_batch;
   int total_tiles;
   int nchunks;
@@ -76,6 +77,9 @@ struct TcArgs {
   int32_t *ids;
   int *err;
   uint32_t idesc;
+  // optional: the counting sort's tile histogram, H[b][row / 2048][id] += 1
+  uint32_t *hist;
+  int hist_tiles;
 };
 
 template <bool RESIDENT, int KB, int STAGES>
@@ -544,7 +548,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int oi = __float_as_int(o.y);
         if (ov > val || (ov == val && oi < idx)) idx = oi;
         const int row = row0 + r_in_tile;
-        if (row < a.N) a.ids[(size_t)b * a.N + row] = idx;
+        if (row < a.N) {
+          a.ids[(size_t)b * a.N + row] = idx;
+          if (a.hist)  // the sort's first kernel, fused: count the id in its sort tile
+            atomicAdd(a.hist + ((size_t)b * a.hist_tiles + row / kSortTile) * a.K + idx, 1u);
+        }
       }
     }
   }
@@ -660,13 +668,16 @@ int launch_point_norms(const void *x, int dtype, long long rows, int d, float *x
 
 int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float *xn, int dtype,
                      int B, long long N, int K, int d, long long Kpad, int32_t *ids, int *err,
-                     cudaStream_t s) {
+                     cudaStream_t s, uint32_t *hist) {
   CUtensorMap tmx, tmc, tme;
   FK_TRY(encode_3d(&tmx, x, dtype, d, N, B, kBlockK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B));
   FK_TRY(encode_3d(&tmc, ch, dtype, d, K, B, kBlockK, kChunkN, CU_TENSOR_MAP_SWIZZLE_128B));
   FK_TRY(encode_3d(&tme, cnx, dtype, kExt, Kpad, B, kExt, kChunkN, CU_TENSOR_MAP_SWIZZLE_32B));
   TcArgs a;
   a.N = (int)N;
+  a.K = K;
+  a.hist = hist;
+  a.hist_tiles = (int)((N + kSortTile - 1) / kSortTile);
   a.tiles_per_batch = (int)((N + kTileM - 1) / kTileM);
   long long total = (long long)B * a.tiles_per_batch;
   if (total > 0x7fffffffLL) return set_error(FK_EUNSUPPORTED, "too many point tiles");

@@ -122,9 +122,12 @@ int launch_assign_f32(const float *x, const float *c, int B, long long N, int K,
 // cnx: extension rows (B, Kpad, 16) in dtype from launch_prep_cn / finalize;
 // xn: ||x||^2 per point (B, N) from launch_point_norms, or NULL (the kernel
 // then computes it from its shared copy of each point tile).
+// hist (nullable, zeroed by the caller, K <= 4096): the counting sort's tile
+// histogram (B, ceil(N / kSortTile), K) is accumulated as the ids are written
+// (run_sort_prehist then skips its histogram kernel).
 int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float *xn, int dtype,
                      int B, long long N, int K, int d, long long Kpad, int32_t *ids, int *err,
-                     cudaStream_t s);
+                     cudaStream_t s, uint32_t *hist = nullptr);
 // xn[r] = ||x_r||^2 (fp32 accumulation) for `rows` rows of d 16-bit elements.
 int launch_point_norms(const void *x, int dtype, long long rows, int d, float *xn, cudaStream_t s);
 
@@ -132,6 +135,12 @@ int launch_point_norms(const void *x, int dtype, long long rows, int d, float *x
 // NULL); perm always written, keys_out (sorted ids) when not NULL.
 int run_sort(Workspace *ws, const int32_t *ids, int B, long long N, int K, int32_t *counts,
              int32_t *offsets, int32_t *perm, int32_t *keys_out, cudaStream_t s);
+// The same single-pass sort (K <= 4096) when ws->table already holds the tile
+// histogram (filled by the assign).  sort_table_bytes: its size.
+bool sort_single_pass(int K);
+size_t sort_table_bytes(int B, long long N, int K);
+int run_sort_prehist(Workspace *ws, const int32_t *ids, int B, long long N, int K, int32_t *counts,
+                     int32_t *offsets, int32_t *perm, int32_t *keys_out, cudaStream_t s);
 
 // segment reduce: owner partials to sums (B, K, d), continuation partials to
 // first (B, pieces_of(N), d).

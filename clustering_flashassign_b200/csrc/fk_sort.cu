@@ -345,15 +345,17 @@ int set_attrs() {
 // offsets_out (B, bins), when not NULL, their exclusive scan.
 int one_pass(Workspace *ws, const int32_t *keys_in, const int32_t *vals_in, int B, int N, int K,
              int T, PassCfg pc, int32_t *digit_counts, int32_t *offsets_out, int32_t *keys_out,
-             int32_t *vals_out, cudaStream_t s) {
+             int32_t *vals_out, cudaStream_t s, bool have_hist = false) {
   FK_TRY(ensure(ws->table, (size_t)B * T * pc.bins * sizeof(uint32_t)));
   uint32_t *H = (uint32_t *)ws->table.p;
   const dim3 grid((unsigned)T, (unsigned)B);
   const size_t shm_h = (size_t)kSortWarps * pc.bins * sizeof(uint32_t);
   const size_t shm_s = (size_t)(kSortWarps + 1) * pc.bins * sizeof(uint32_t);
-  k_tile_hist<<<grid, kSortThreads, shm_h, s>>>(keys_in, N, K, T, pc, H, ws->err);
-  count_launch();
-  FK_CUDA(cudaGetLastError());
+  if (!have_hist) {
+    k_tile_hist<<<grid, kSortThreads, shm_h, s>>>(keys_in, N, K, T, pc, H, ws->err);
+    count_launch();
+    FK_CUDA(cudaGetLastError());
+  }
   k_scan_tiles<<<dim3((unsigned)((pc.bins + 31) / 32), (unsigned)B), kSortThreads, 0, s>>>(
       H, pc.bins, T, digit_counts);
   count_launch();
@@ -366,6 +368,31 @@ int one_pass(Workspace *ws, const int32_t *keys_in, const int32_t *vals_in, int 
 }
 
 }  // namespace
+
+bool sort_single_pass(int K) { return bits_for(K) <= kMaxDigitBits; }
+
+size_t sort_table_bytes(int B, long long N, int K) {
+  return (size_t)B * ((N + kSortTile - 1) / kSortTile) * K * sizeof(uint32_t);
+}
+
+int run_sort_prehist(Workspace *ws, const int32_t *ids, int B, long long N_, int K, int32_t *counts,
+                     int32_t *offsets, int32_t *perm, int32_t *keys_out, cudaStream_t s) {
+  if (!sort_single_pass(K)) return set_error(FK_EUNSUPPORTED, "fused histogram needs K <= 4096");
+  FK_TRY(set_attrs());
+  const int N = (int)N_;
+  const int T = (int)((N_ + kSortTile - 1) / kSortTile);
+  int32_t *cnt = counts, *off = offsets;
+  if (!cnt) {
+    FK_TRY(ensure(ws->counts, (size_t)B * K * sizeof(int32_t)));
+    cnt = (int32_t *)ws->counts.p;
+  }
+  if (!off) {
+    FK_TRY(ensure(ws->offsets, (size_t)B * K * sizeof(int32_t)));
+    off = (int32_t *)ws->offsets.p;
+  }
+  PassCfg pc{0, 0xffffffffu, K, bits_for(K), true};
+  return one_pass(ws, ids, nullptr, B, N, K, T, pc, cnt, off, keys_out, perm, s, true);
+}
 
 int run_sort(Workspace *ws, const int32_t *ids, int B, long long N_, int K, int32_t *counts,
              int32_t *offsets, int32_t *perm, int32_t *keys_out, cudaStream_t s) {
