@@ -495,7 +495,9 @@ def run_largen(args):
 
 def run_kernel_case(args):
     """Launch only one step kind on the bench workload (for profiler captures):
-    assign = fk_assign, update = fk_update, each warmup + steps times."""
+    assign = fk_assign, update = fk_update, lloyd = fk_lloyd with two
+    iterations (its assign uses the precomputed point norms and fills the
+    sort's tile histogram, as in the bench), each warmup + steps times."""
     import torch
 
     import clustering_flashassign_b200 as fk
@@ -514,6 +516,8 @@ def run_kernel_case(args):
     for _ in range(args.warmup + args.steps):
         if args.kernel_case == "assign":
             fk.fk_assign(xd, cd, ids)
+        elif args.kernel_case == "lloyd":
+            fk.fk_lloyd(xd, cd, 2, 0.0, ids, centers)
         else:
             fk.fk_update(xd, ids, centers, counts)
     torch.cuda.synchronize()
@@ -527,7 +531,7 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="fk", choices=["fk", "reference"])
-    ap.add_argument("--kernel-case", default=None, choices=["assign", "update"],
+    ap.add_argument("--kernel-case", default=None, choices=["assign", "update", "lloyd"],
                     help="launch only this step (profiler captures); prints no bench line")
     ap.add_argument("--points", type=int, default=0, help="with --kernel-case / --workload: points per batch")
     ap.add_argument("--workload", default="api", choices=["api", "tiny", "zipf", "splitd", "largen"],
