@@ -144,6 +144,8 @@ constexpr int kSliceBytes = 256;                        // 128 x 16-bit elements
 constexpr int kBatches = kPiece / kRowsPerBatch;        // 8
 constexpr int kKeyChunks = kPiece / 32;                 // 4
 constexpr int kBufBytes = kRowsPerBatch * kSliceBytes;  // 4 KB per batch buffer
+// the batch loop below pairs two batches per 32-position key chunk
+static_assert(2 * kRowsPerBatch == 32, "k_segreduce16 assumes two 16-row batches per key chunk");
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool ok) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(ok ? 16 : 0)
