@@ -159,3 +159,30 @@ def test_repeated_runs_are_bit_identical():
         outs.append((ids, cen))
     assert torch.equal(outs[0][0], outs[1][0])
     assert torch.equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("tol_iters", [2, 3])
+def test_tol_stop_returns_the_same_state_as_a_fixed_run(tol_iters):
+    """The assign of the next iteration is queued before the host reads the
+    shift; when the shift stops the loop that assign must not leak: ids and
+    centroids equal those of a run with exactly that many iterations."""
+    import clustering_flashassign_b200 as fk
+    B, N, K, d = 2, 3000, 12, 32
+    x, idx, c0 = case(B, N, K, d, "f16", n_comp=12, mean_std=25.0)
+    xd, cd = to_dev(x, "f16"), to_dev(c0, "f16")
+    ids_f = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    cen_f = torch.empty((B, K, d), dtype=torch.float32, device="cuda")
+    # max centroid shift of iteration n (n >= 2) from fixed runs of n - 1 and n iterations
+    cens = []
+    for n in range(1, tol_iters + 1):
+        fk.fk_lloyd(xd, cd, n, 0.0, ids_f, cen_f)
+        cens.append(cen_f.clone())
+    s_stop = float((cens[-1] - cens[-2]).norm(dim=-1).max())
+    tol = s_stop * 1.0001  # the run stops at iteration tol_iters, or earlier
+    ids_t = torch.empty_like(ids_f)
+    cen_t = torch.empty_like(cen_f)
+    n = fk.fk_lloyd(xd, cd, 20, tol, ids_t, cen_t)
+    fk.fk_lloyd(xd, cd, n, 0.0, ids_f, cen_f)
+    assert n <= tol_iters
+    assert torch.equal(ids_t, ids_f)
+    assert torch.equal(cen_t, cen_f)
