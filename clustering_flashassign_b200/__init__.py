@@ -29,7 +29,7 @@ DTYPES = {torch.float32: FK_F32, torch.float16: FK_F16, torch.bfloat16: FK_BF16}
 
 EXPORTS = ["fk_assign", "fk_update", "fk_sort", "fk_lloyd", "fk_assign_noalloc", "fk_status_string",
            "fk_last_error", "fk_device_error", "fk_release", "fk_profile_enable", "fk_profile_read",
-           "fk_launch_count", "fk_version"]
+           "fk_launch_count", "fk_version", "fk_selftest_bounded_wait"]
 
 
 class FkError(RuntimeError):
@@ -75,6 +75,7 @@ def _load():
         "fk_profile_read": (I, [ctypes.POINTER(FkProfile), I]),
         "fk_launch_count": (LL, []),
         "fk_version": (I, []),
+        "fk_selftest_bounded_wait": (I, [LL, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -168,6 +169,11 @@ def fk_lloyd(x: torch.Tensor, init_centers: torch.Tensor, max_iter: int, tol: fl
 
 def fk_device_error(stream=None) -> int:
     return int(lib.fk_device_error(_stream(stream)))
+
+
+def fk_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
+    """Status of a kernel whose mbarrier wait can never complete (FK_ETIMEOUT expected)."""
+    return int(lib.fk_selftest_bounded_wait(ctypes.c_longlong(int(limit_ns)), _stream(stream)))
 
 
 def fk_release() -> None:

@@ -209,6 +209,16 @@ const char *fk_last_error(void);
  */
 int fk_device_error(fk_stream_t stream);
 
+/*
+ * fk_selftest_bounded_wait -- a check of the failure path, not part of the
+ * method (the pages have no counterpart).  Launches one CTA that waits on an
+ * mbarrier nothing ever arrives at, with the same bounded wait loop as the
+ * tcgen05 kernels but a limit of limit_ns nanoseconds (0 < limit_ns <= 1e10).
+ * Returns FK_ETIMEOUT (read from the device error word, which is then clear)
+ * when the bounded wait works; the CUDA context stays usable.
+ */
+int fk_selftest_bounded_wait(long long limit_ns, fk_stream_t stream);
+
 /* Frees every workspace of the current device (no call may be in flight). */
 int fk_release(void);
 

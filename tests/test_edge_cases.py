@@ -111,3 +111,21 @@ def test_k_equals_n_two_pass_sort_and_update():
     np.testing.assert_array_equal(counts.cpu().numpy(), rc)
     check_centers(cen.cpu().numpy(), new, "f16")
     assert fk.fk_device_error() == 0
+
+
+def test_bounded_wait_expires_and_the_context_survives():
+    """A kernel whose mbarrier wait can never complete gives up after its
+    limit and reports FK_ETIMEOUT; later calls on the same context work."""
+    import time
+
+    import clustering_flashassign_b200 as fk
+    t0 = time.perf_counter()
+    st = fk.fk_selftest_bounded_wait(20_000_000)  # 20 ms
+    dt = time.perf_counter() - t0
+    assert st == fk.FK_ETIMEOUT
+    assert 0.015 < dt < 5.0
+    assert fk.fk_device_error() == 0  # the word was read and cleared
+    x, _, c = case(1, 500, 40, 64, "f16", seed=23)
+    g, err = _assign(x, c, "f16")
+    assert err == 0
+    check_ids(g, x, "f16", synthdata.to_f64(c, "f16"))
