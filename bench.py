@@ -493,6 +493,79 @@ def run_largen(args):
     print(json.dumps(line), flush=True)
 
 
+def run_baselines(args):
+    """The pages' comparison points, rebuilt on B200 at the api shape (context
+    for the kernels' speedups; library code, not the product path):
+      - assign with the distance matrix materialised: one cuBLAS batched GEMM
+        writes D = ||c||^2 - 2 X C^T (B, N, K) in fp16, then an argmin reads it;
+      - update by scatter atomics: index_add_ of every point row (fp32) into its
+        centroid's sum, a bincount, a division.
+    Both are timed with CUDA events next to fk_assign and fk_update on the same
+    inputs (the fp32 copy of the points for index_add_ is made outside the
+    timed region)."""
+    import torch
+
+    import clustering_flashassign_b200 as fk
+    w, x, init = make_inputs(0)
+    dev = torch.device("cuda", 0)
+    xd = torch.from_numpy(x).to(dev)
+    cd = torch.from_numpy(init).to(dev)
+    B, N, K, d = w.B, w.N, w.K, w.d
+
+    def timed(fn, reps):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    cn = (cd.float() ** 2).sum(-1).half().unsqueeze(1)  # (B, 1, K)
+    ct = cd.transpose(1, 2).contiguous()                 # (B, d, K)
+    ids_ref = torch.empty((B, N), dtype=torch.int64, device=dev)
+
+    def assign_matd():
+        dmat = torch.baddbmm(cn, xd, ct, alpha=-2.0)     # (B, N, K) fp16 in HBM
+        torch.argmin(dmat, dim=2, out=ids_ref)
+
+    ids = torch.empty((B, N), dtype=torch.int32, device=dev)
+    t_matd = timed(assign_matd, args.steps)
+    t_fa = timed(lambda: fk.fk_assign(xd, cd, ids), args.steps)
+    agree = float((ids.long() == ids_ref).float().mean())
+
+    x32 = xd.float().view(B * N, d)
+    flat = (ids.long() + torch.arange(B, device=dev).unsqueeze(1) * K).view(-1)
+    sums = torch.zeros((B * K, d), dtype=torch.float32, device=dev)
+
+    def update_scatter():
+        sums.zero_()
+        sums.index_add_(0, flat, x32)
+        cnt = torch.bincount(flat, minlength=B * K).clamp_min(1)
+        return sums / cnt.unsqueeze(1)
+
+    centers = cd.float()
+    counts = torch.empty((B, K), dtype=torch.int32, device=dev)
+    t_scat = timed(update_scatter, args.steps)
+    t_upd = timed(lambda: fk.fk_update(xd, ids, centers.clone(), counts), args.steps)
+    flop = 2.0 * B * N * K * d
+    line = {
+        "metric": "baselines at the api shape (ms per call; ratio = baseline / libfk)",
+        "workload": f"api: B={B} N={N} K={K} d={d} {w.dtype}",
+        "assign_materialised_d_ms": t_matd, "assign_flashassign_ms": t_fa,
+        "assign_ratio": t_matd / t_fa, "assign_ids_agree": agree,
+        "materialised_d_bytes": B * N * K * 2,
+        "update_scatter_atomic_ms": t_scat, "update_sort_inverse_ms": t_upd,
+        "update_ratio": t_scat / t_upd,
+        "scatter_atomic_gbs": B * N * d * 4 / (t_scat * 1e-3) / 1e9,
+        "flashassign_tflops": flop / (t_fa * 1e-3) / 1e12,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_kernel_case(args):
     """Launch only one step kind on the bench workload (for profiler captures):
     assign = fk_assign, update = fk_update, lloyd = fk_lloyd with two
@@ -534,6 +607,8 @@ def main():
     ap.add_argument("--kernel-case", default=None, choices=["assign", "update", "lloyd"],
                     help="launch only this step (profiler captures); prints no bench line")
     ap.add_argument("--points", type=int, default=0, help="with --kernel-case / --workload: points per batch")
+    ap.add_argument("--baselines", action="store_true",
+                    help="time the materialised-distance assign and the scatter-atomic update next to libfk")
     ap.add_argument("--workload", default="api", choices=["api", "tiny", "zipf", "splitd", "largen"],
                     help="api is the benchmark; the others print their own line (largen: the 64 GiB "
                          "streamed workload)")
@@ -546,6 +621,9 @@ def main():
         return
     if args.kernel_case:
         run_kernel_case(args)
+        return
+    if args.baselines:
+        run_baselines(args)
         return
     if args.workload == "largen":
         run_largen(args)
