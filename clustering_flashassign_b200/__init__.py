@@ -52,7 +52,7 @@ class FkProfile(ctypes.Structure):
     _fields_ = [("assign_ms", ctypes.c_double), ("assign_launches", ctypes.c_longlong),
                 ("sort_ms", ctypes.c_double), ("reduce_ms", ctypes.c_double),
                 ("finalize_ms", ctypes.c_double), ("update_calls", ctypes.c_longlong),
-                ("kernel_launches", ctypes.c_longlong)]
+                ("kernel_launches", ctypes.c_longlong), ("update_ms", ctypes.c_double)]
 
 
 def _load():
@@ -180,8 +180,9 @@ def fk_release() -> None:
     _check(lib.fk_release(), "fk_release")
 
 
-def fk_profile_enable(on: bool = True) -> None:
-    _check(lib.fk_profile_enable(1 if on else 0), "fk_profile_enable")
+def fk_profile_enable(on=True) -> None:
+    """0 / False: off; 1 / True: every phase; 2: assign and whole update only."""
+    _check(lib.fk_profile_enable(int(on)), "fk_profile_enable")
 
 
 def fk_profile_read(reset: bool = False) -> dict:

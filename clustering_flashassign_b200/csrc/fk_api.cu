@@ -76,6 +76,7 @@ int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long
               int dtype, float *centers, int32_t *counts_out, void *ch, void *cnx, long long Kpad,
               cudaStream_t s, bool have_hist = false) {
   note_update_call();
+  PhaseTimer whole(PH_UPDATE, s);
   int32_t *counts = counts_out;
   if (!counts) {
     FK_TRY(ensure(ws->counts, (size_t)B * K * sizeof(int32_t)));

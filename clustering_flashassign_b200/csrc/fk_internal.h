@@ -78,7 +78,7 @@ int workspace_for(cudaStream_t s, Workspace **out);
 
 // Launch accounting and event timing.
 void count_launch(int n = 1);
-enum Phase { PH_ASSIGN = 0, PH_SORT = 1, PH_REDUCE = 2, PH_FINALIZE = 3 };
+enum Phase { PH_ASSIGN = 0, PH_SORT = 1, PH_REDUCE = 2, PH_FINALIZE = 3, PH_UPDATE = 4, PH_COUNT = 5 };
 struct PhaseTimer {
   cudaEvent_t a = nullptr, b = nullptr;
   int phase;

@@ -17,13 +17,14 @@ std::map<std::pair<int, cudaStream_t>, Workspace *> g_ws;
 std::atomic<long long> g_launches{0};
 
 std::mutex g_prof_mu;
-bool g_prof_on = false;
+int g_prof_level = 0;  // 0 off, 1 every phase, 2 assign + whole update
+std::vector<cudaEvent_t> g_event_pool;  // recorded events are reused, not recreated
 struct Pending {
   cudaEvent_t a, b;
   int phase;
 };
 std::vector<Pending> g_pending;
-double g_ms[4] = {0, 0, 0, 0};
+double g_ms[PH_COUNT] = {0, 0, 0, 0, 0};
 long long g_assign_launches = 0, g_update_calls = 0, g_prof_launches = 0;
 }  // namespace
 
@@ -126,7 +127,7 @@ int release_device_workspaces() {
 
 void count_launch(int n) {
   g_launches.fetch_add(n, std::memory_order_relaxed);
-  if (g_prof_on) {
+  if (g_prof_level) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     g_prof_launches += n;
   }
@@ -134,9 +135,28 @@ void count_launch(int n) {
 
 long long launch_count() { return g_launches.load(); }
 
+namespace {
+cudaEvent_t take_event() {
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (!g_event_pool.empty()) {
+      cudaEvent_t e = g_event_pool.back();
+      g_event_pool.pop_back();
+      return e;
+    }
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+}  // namespace
+
 PhaseTimer::PhaseTimer(int ph, cudaStream_t st) : phase(ph), s(st) {
-  if (!g_prof_on) return;
-  if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) {
+  if (!g_prof_level) return;
+  if (g_prof_level == 2 && ph != PH_ASSIGN && ph != PH_UPDATE) return;
+  a = take_event();
+  b = take_event();
+  if (!a || !b) {
     a = b = nullptr;
     return;
   }
@@ -152,13 +172,14 @@ PhaseTimer::~PhaseTimer() {
 }
 
 void note_update_call() {
-  if (!g_prof_on) return;
+  if (!g_prof_level) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
   ++g_update_calls;
 }
 
 int profile_enable(int on) {
-  g_prof_on = on != 0;
+  if (on < 0 || on > 2) return set_error(FK_EINVAL, "profile level must be 0, 1 or 2");
+  g_prof_level = on;
   return FK_OK;
 }
 
@@ -168,8 +189,8 @@ int profile_read(fk_profile *out, int reset) {
     float ms = 0.f;
     cudaEventSynchronize(p.b);
     if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) g_ms[p.phase] += ms;
-    cudaEventDestroy(p.a);
-    cudaEventDestroy(p.b);
+    g_event_pool.push_back(p.a);
+    g_event_pool.push_back(p.b);
   }
   g_pending.clear();
   if (out) {
@@ -177,6 +198,7 @@ int profile_read(fk_profile *out, int reset) {
     out->sort_ms = g_ms[PH_SORT];
     out->reduce_ms = g_ms[PH_REDUCE];
     out->finalize_ms = g_ms[PH_FINALIZE];
+    out->update_ms = g_ms[PH_UPDATE];
     out->assign_launches = g_assign_launches;
     out->update_calls = g_update_calls;
     out->kernel_launches = g_prof_launches;

@@ -231,9 +231,12 @@ typedef struct {
   double finalize_ms; /* divide / shift / dtype copy kernel */
   long long update_calls;
   long long kernel_launches; /* every kernel this library launched while enabled */
+  double update_ms;   /* whole update calls (sort + reduce + finalize, gaps included) */
 } fk_profile;
 
-/* Turns event timing on (1) or off (0).  Off by default. */
+/* Event timing: 0 off (default), 1 every phase (assign, sort, reduce,
+ * finalize, whole update), 2 light (assign and whole update only: two event
+ * pairs per Lloyd iteration). */
 int fk_profile_enable(int on);
 
 /* Synchronizes the recorded events, fills *out, and clears the totals if reset != 0. */
