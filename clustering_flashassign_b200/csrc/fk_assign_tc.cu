@@ -88,8 +88,14 @@ struct Layout {
   static constexpr uint32_t kAExtOff = kXBytes;
   static constexpr uint32_t kAExtTotal = RESIDENT ? 2u * kAExtBytes : kAExtBytes;
   static constexpr uint32_t kBExtOff = kAExtOff + kAExtTotal;
-  static constexpr uint32_t kStagesOff = kBExtOff + kExtSlots * kBExtBytes;
-  static constexpr uint32_t kStageBytes = RESIDENT ? kCBlockBytes : kXBlockBytes + kCBlockBytes;
+  // resident: a stage holds a whole chunk (its KB centroid K-blocks and its
+  // norm rows), so the MMA thread waits and commits once per chunk; split-d:
+  // a stage holds one 64-wide K-block of points and centroids, and the norm
+  // rows have their own ring.
+  static constexpr int kRing = RESIDENT ? 0 : kExtSlots;
+  static constexpr uint32_t kStagesOff = kBExtOff + kRing * kBExtBytes;
+  static constexpr uint32_t kStageBytes =
+      RESIDENT ? KB * kCBlockBytes + kBExtBytes : kXBlockBytes + kCBlockBytes;
   static constexpr uint32_t kBarOff = kStagesOff + STAGES * kStageBytes;
   // barriers: full[S], empty[S], efull[E], eempty[E], xfull[2], xempty[2],
   //           xnfull[2], accfull[2], accempty[2], mfull[2], mempty[2], drain
@@ -298,25 +304,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = tile / a.tiles_per_batch;
         const int row0 = (tile % a.tiles_per_batch) * kTileM;
         for (int c = 0; ok && c < a.nchunks; ++c) {
-          {  // this chunk's centroid norm rows (used by the chunk's last MMA step)
+          if (RESIDENT) {  // the whole chunk and its norm rows in one stage
+            const int s = f % STAGES;
+            if (!mbar_wait(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+            const uint32_t dst = st_base + s * L::kStageBytes;
+            mbar_arrive_expect_tx(full(s), L::kStageBytes);
+            for (int kb = 0; kb < KB; ++kb)
+              tma_load_3d(&tmc, dst + kb * kCBlockBytes, full(s), kb * kBlockK, c * kChunkN, b);
+            tma_load_3d(&tme, dst + KB * kCBlockBytes, full(s), 0, c * kChunkN, b);
+            ++f;
+          } else {  // this chunk's centroid norm rows (used by the chunk's last MMA step)
             const int es = e % kExtSlots;
             if (!mbar_wait(eempty(es), ((e / kExtSlots) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
             mbar_arrive_expect_tx(efull(es), kBExtBytes);
             tma_load_3d(&tme, bext_base + es * kBExtBytes, efull(es), 0, c * kChunkN, b);
             ++e;
           }
-          for (int kb = 0; kb < kblocks; ++kb) {
+          for (int kb = 0; !RESIDENT && kb < kblocks; ++kb) {
             const int s = f % STAGES;
             if (!mbar_wait(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
             const uint32_t dst = st_base + s * L::kStageBytes;
-            if (RESIDENT) {
-              mbar_arrive_expect_tx(full(s), kCBlockBytes);
-              tma_load_3d(&tmc, dst, full(s), kb * kBlockK, c * kChunkN, b);
-            } else {
-              mbar_arrive_expect_tx(full(s), kXBlockBytes + kCBlockBytes);
-              tma_load_3d(&tmx, dst, full(s), kb * kBlockK, row0, b);
-              tma_load_3d(&tmc, dst + kXBlockBytes, full(s), kb * kBlockK, c * kChunkN, b);
-            }
+            mbar_arrive_expect_tx(full(s), kXBlockBytes + kCBlockBytes);
+            tma_load_3d(&tmx, dst, full(s), kb * kBlockK, row0, b);
+            tma_load_3d(&tmc, dst + kXBlockBytes, full(s), kb * kBlockK, c * kChunkN, b);
             ++f;
           }
           if (RESIDENT && ok && c == 0 && tile + (int)gridDim.x < a.total_tiles)
@@ -353,6 +363,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(accempty(ab), ((h >> 1) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem + ab * kChunkN;
+          if (RESIDENT) {
+            if (c == 0) {  // the tile's point norm rows are written
+              if (!mbar_wait(xnfull(xb), (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+            }
+            const int s = f % STAGES;
+            if (!mbar_wait(full(s), (f / STAGES) & 1, abort_flag, a.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t stage = st_base + s * L::kStageBytes;
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) {
+              const uint32_t a_addr = x_base + (xb * KB + kb) * kXBlockBytes;
+              const uint32_t b_addr = stage + kb * kCBlockBytes;
+#pragma unroll
+              for (int k = 0; k < kBlockK / 16; ++k)
+                mma_f16(d_tmem, desc_k_sw128(a_addr + k * 32), desc_k_sw128(b_addr + k * 32), a.idesc,
+                        (kb | k) != 0 ? 1u : 0u);
+            }
+            // the norm step: acc += A_ext . B_ext (fk_norms.cuh)
+            mma_f16(d_tmem, desc_k_sw32(a_ext), desc_k_sw32(stage + KB * kCBlockBytes), a.idesc, 1u);
+            mma_commit(empty(s));  // frees the stage once these MMAs have read it
+            ++f;
+            mma_commit(accfull(ab));  // accumulator ready for the epilogue
+            ++h;
+            continue;
+          }
           for (int kb = 0; kb < kblocks; ++kb) {
             const int s = f % STAGES;
             if (!mbar_wait(full(s), (f / STAGES) & 1, abort_flag, a.err)) { ok = false; break; }
@@ -654,8 +689,9 @@ int launch_variant(const CUtensorMap &tmx, const CUtensorMap &tmc, const CUtenso
 template <typename T>
 int launch_typed(const CUtensorMap &tmx, const CUtensorMap &tmc, const CUtensorMap &tme,
                  const TcArgs &a, int grid, cudaStream_t s) {
-  if (a.kblocks == 1) return launch_variant<T, true, 1, 5>(tmx, tmc, tme, a, grid, s);
-  if (a.kblocks == 2) return launch_variant<T, true, 2, 4>(tmx, tmc, tme, a, grid, s);
+  // resident stages hold whole chunks: 4 x 40 KB (d <= 64) or 2 x 72 KB (d <= 128)
+  if (a.kblocks == 1) return launch_variant<T, true, 1, 4>(tmx, tmc, tme, a, grid, s);
+  if (a.kblocks == 2) return launch_variant<T, true, 2, 2>(tmx, tmc, tme, a, grid, s);
   return launch_variant<T, false, 1, 4>(tmx, tmc, tme, a, grid, s);
 }
 
