@@ -55,13 +55,12 @@ int read_device_error(Workspace *ws, cudaStream_t s) {
   return set_error(FK_EINVAL, "an id outside [0, K) reached the update");
 }
 
-// Scratch of one update over B batches of n sorted positions: sorted keys,
-// perm, segment offsets, owner partial sums (B, K, d) and continuation
+// Scratch of one update over B batches of n sorted positions: sorted
+// (id, point) pairs, segment offsets, owner partial sums (B, K, d) and continuation
 // partials (B, pieces, d).  Nothing here needs clearing: every value read is
 // written by the same update first.
 int prepare_update(Workspace *ws, int B, long long n, int K, int d) {
-  FK_TRY(ensure(ws->keys_a, (size_t)B * n * sizeof(int32_t)));
-  FK_TRY(ensure(ws->vals_a, (size_t)B * n * sizeof(int32_t)));
+  FK_TRY(ensure(ws->kv, (size_t)B * n * sizeof(int2)));
   FK_TRY(ensure(ws->offsets, (size_t)B * K * sizeof(int32_t)));
   FK_TRY(ensure(ws->sums, (size_t)B * K * d * sizeof(float)));
   FK_TRY(ensure(ws->first, (size_t)B * pieces_of(n) * d * sizeof(float)));
@@ -84,17 +83,17 @@ int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long
   }
   FK_TRY(prepare_update(ws, B, N, K, d));
   FK_CUDA(cudaMemsetAsync(ws->maxshift, 0, sizeof(unsigned), s));
-  int32_t *keys = (int32_t *)ws->keys_a.p, *perm = (int32_t *)ws->vals_a.p;
+  int2 *kv = (int2 *)ws->kv.p;
   int32_t *offsets = (int32_t *)ws->offsets.p;
   float *sums = (float *)ws->sums.p, *first = (float *)ws->first.p;
   {
     PhaseTimer t(PH_SORT, s);
-    if (have_hist) FK_TRY(run_sort_prehist(ws, ids, B, N, K, counts, offsets, perm, keys, s));
-    else FK_TRY(run_sort(ws, ids, B, N, K, counts, offsets, perm, keys, s));
+    if (have_hist) FK_TRY(run_sort_prehist(ws, ids, B, N, K, counts, offsets, nullptr, kv, s));
+    else FK_TRY(run_sort(ws, ids, B, N, K, counts, offsets, nullptr, kv, s));
   }
   {
     PhaseTimer t(PH_REDUCE, s);
-    FK_TRY(launch_segreduce(x, dtype, keys, perm, B, N, K, d, sums, first, s));
+    FK_TRY(launch_segreduce(x, dtype, kv, B, N, K, d, sums, first, s));
   }
   PhaseTimer t(PH_FINALIZE, s);
   return launch_finalize(sums, first, pieces_of(N), counts, offsets, centers, ch, cnx, dtype, B, K,
@@ -163,7 +162,7 @@ int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void
   FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cnx, ws->err, s));
   FK_TRY(prepare_update(ws, 1, chunk, K, d));
   float *sums = (float *)ws->sums.p, *first = (float *)ws->first.p;
-  int32_t *keys = (int32_t *)ws->keys_a.p, *perm = (int32_t *)ws->vals_a.p;
+  int2 *kv = (int2 *)ws->kv.p;
   int32_t *offsets = (int32_t *)ws->offsets.p;
   long long job = 0;
   int it = 0;
@@ -190,11 +189,11 @@ int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void
                                   Kpad, idc, s));
         {
           PhaseTimer t(PH_SORT, s);
-          FK_TRY(run_sort(ws, idc, 1, nc, K, counts, offsets, perm, keys, s));
+          FK_TRY(run_sort(ws, idc, 1, nc, K, counts, offsets, nullptr, kv, s));
         }
         {
           PhaseTimer t(PH_REDUCE, s);
-          FK_TRY(launch_segreduce(xb, dtype, keys, perm, 1, nc, K, d, sums, first, s));
+          FK_TRY(launch_segreduce(xb, dtype, kv, 1, nc, K, d, sums, first, s));
           FK_TRY(launch_accumulate(sums, first, pieces_of(nc), counts, offsets, K, d,
                                    gsum + (size_t)b * K * d, gcounts + (size_t)b * K, s));
         }

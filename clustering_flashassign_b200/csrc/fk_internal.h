@@ -52,7 +52,7 @@ struct Workspace {
   int *err = nullptr;             // device error word
   unsigned *maxshift = nullptr;   // device, float bits (non-negative floats order as uints)
   float *h_maxshift = nullptr;    // pinned host mirror
-  DevBuf cn, ch, sums, first, counts, offsets, table, digit_off, keys_a, vals_a, keys_b, vals_b;
+  DevBuf cn, ch, sums, first, counts, offsets, table, digit_off, kv, keys_b, vals_b;
   DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2], gsum, gcounts, xn, ids_alt;
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
@@ -132,19 +132,20 @@ int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float
 int launch_point_norms(const void *x, int dtype, long long rows, int d, float *xn, cudaStream_t s);
 
 // counting sort: counts / offsets optional (workspace offsets are used when
-// NULL); perm always written, keys_out (sorted ids) when not NULL.
+// NULL); perm (sorted position -> point) and kv_out (sorted (id, point) pairs)
+// are each written when not NULL.
 int run_sort(Workspace *ws, const int32_t *ids, int B, long long N, int K, int32_t *counts,
-             int32_t *offsets, int32_t *perm, int32_t *keys_out, cudaStream_t s);
+             int32_t *offsets, int32_t *perm, int2 *kv_out, cudaStream_t s);
 // The same single-pass sort (K <= 4096) when ws->table already holds the tile
 // histogram (filled by the assign).  sort_table_bytes: its size.
 bool sort_single_pass(int K);
 size_t sort_table_bytes(int B, long long N, int K);
 int run_sort_prehist(Workspace *ws, const int32_t *ids, int B, long long N, int K, int32_t *counts,
-                     int32_t *offsets, int32_t *perm, int32_t *keys_out, cudaStream_t s);
+                     int32_t *offsets, int32_t *perm, int2 *kv_out, cudaStream_t s);
 
-// segment reduce: owner partials to sums (B, K, d), continuation partials to
-// first (B, pieces_of(N), d).
-int launch_segreduce(const void *x, int dtype, const int32_t *skeys, const int32_t *perm, int B,
-                     long long N, int K, int d, float *sums, float *first, cudaStream_t s);
+// segment reduce over the sorted (id, point) pairs kv (B, N): owner partials
+// to sums (B, K, d), continuation partials to first (B, pieces_of(N), d).
+int launch_segreduce(const void *x, int dtype, const int2 *kv, int B, long long N, int K, int d,
+                     float *sums, float *first, cudaStream_t s);
 
 }  // namespace fk

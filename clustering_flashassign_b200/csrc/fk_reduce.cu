@@ -1,7 +1,7 @@
 // Segment reduction of the sort-inverse update (step a5, before finalize).
 //
-// After the counting sort, equal ids are contiguous: skeys[b][j] is the id at
-// sorted position j and perm[b][j] the point index there.  The points are
+// After the counting sort, equal ids are contiguous: kv[b][j] = (id, point)
+// holds the id at sorted position j and the index of the point there.  The points are
 // never moved; rows are gathered in sorted order and each run of equal ids is
 // reduced on chip in fp32 ("Flash-KMeans: IO感知的精确K-Means", section
 // "它攻克的兩大瓶頸": every thread block reduces a segment on chip and issues
@@ -56,8 +56,7 @@ template <> __device__ __forceinline__ void store<1>(float *dst, const float (&a
 
 template <typename T, int VEC>
 __global__ void __launch_bounds__(kWarps * 32) k_segreduce(const T *__restrict__ x,
-                                                           const int32_t *__restrict__ skeys,
-                                                           const int32_t *__restrict__ perm, int N,
+                                                           const int2 *__restrict__ kv, int N,
                                                            int K, int d, int pieces, int colblocks,
                                                            long long items, float *__restrict__ sums,
                                                            float *__restrict__ first) {
@@ -72,12 +71,11 @@ __global__ void __launch_bounds__(kWarps * 32) k_segreduce(const T *__restrict__
   const bool active = c0 < d;
   const int j0 = piece * kPiece;
   const int j1 = min(N, j0 + kPiece);
-  const int32_t *kb = skeys + (size_t)b * N;
-  const int32_t *pb = perm + (size_t)b * N;
+  const int2 *kvb = kv + (size_t)b * N;
   const T *xb = x + (size_t)b * N * d + c0;
   float *sb = sums + (size_t)b * K * d + c0;
   float *fb = first + ((size_t)b * pieces + piece) * d + c0;
-  const int prev = j0 > 0 ? kb[j0 - 1] : -1;
+  const int prev = j0 > 0 ? kvb[j0 - 1].x : -1;
 
   float acc[VEC];
 #pragma unroll
@@ -92,8 +90,9 @@ __global__ void __launch_bounds__(kWarps * 32) k_segreduce(const T *__restrict__
   } while (0)
   for (int jb = j0; jb < j1; jb += 32) {
     const int n = min(32, j1 - jb);
-    int mk = lane < n ? kb[jb + lane] : -1;
-    int mr = lane < n ? pb[jb + lane] : 0;
+    const int2 p = lane < n ? kvb[jb + lane] : make_int2(-1, 0);
+    int mk = p.x;
+    const int mr = p.y;
     // ids must be in [0, K) and rows in [0, N); anything else (left behind by
     // an out-of-range caller id) is skipped
     if ((unsigned)mk >= (unsigned)K || (unsigned)mr >= (unsigned)N) mk = -1;
@@ -187,8 +186,7 @@ __device__ __forceinline__ void add_row(float (&acc)[4], const uint8_t *slice) {
 
 template <typename T>
 __global__ void __launch_bounds__(kWarps * 32) k_segreduce16(const T *__restrict__ x,
-                                                             const int32_t *__restrict__ skeys,
-                                                             const int32_t *__restrict__ perm, int N,
+                                                             const int2 *__restrict__ kv, int N,
                                                              int K, int d, int pieces, int colblocks,
                                                              long long items, float *__restrict__ sums,
                                                              float *__restrict__ first) {
@@ -206,8 +204,7 @@ __global__ void __launch_bounds__(kWarps * 32) k_segreduce16(const T *__restrict
   const int j0 = piece * kPiece;
   const int j1 = min(N, j0 + kPiece);
   const int nb = (j1 - j0 + kRowsPerBatch - 1) / kRowsPerBatch;
-  const int32_t *kb = skeys + (size_t)b * N;
-  const int32_t *pb = perm + (size_t)b * N;
+  const int2 *kvb = kv + (size_t)b * N;
   const T *xb = x + (size_t)b * N * d;
   float *sb = sums + (size_t)b * K * d + c0;
   float *fb = first + ((size_t)b * pieces + piece) * d + c0;
@@ -219,13 +216,14 @@ __global__ void __launch_bounds__(kWarps * 32) k_segreduce16(const T *__restrict
 #pragma unroll
   for (int t = 0; t < kKeyChunks; ++t) {
     const int j = j0 + 32 * t + lane;
-    mk[t] = j < j1 ? kb[j] : -1;
-    mr[t] = j < j1 ? pb[j] : 0;
+    const int2 p = j < j1 ? kvb[j] : make_int2(-1, 0);
+    mk[t] = p.x;
+    mr[t] = p.y;
     // ids must be in [0, K) and rows in [0, N); anything else (left behind by
     // an out-of-range caller id) is skipped
     if ((unsigned)mk[t] >= (unsigned)K || (unsigned)mr[t] >= (unsigned)N) mk[t] = -1;
   }
-  const int prev = j0 > 0 ? kb[j0 - 1] : -1;
+  const int prev = j0 > 0 ? kvb[j0 - 1].x : -1;
   issue_batch<T>(buf, xb, d, col_base, mk[0], mr[0], 0, lane);
   if (nb > 1) issue_batch<T>(buf + kBufBytes, xb, d, col_base, mk[0], mr[0], 1, lane);
 
@@ -291,8 +289,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_segreduce16(const T *__restrict
 }
 
 template <typename T>
-int launch16(const void *x, const int32_t *skeys, const int32_t *perm, int B, int N, int K, int d,
-             float *sums, float *first, cudaStream_t s) {
+int launch16(const void *x, const int2 *kv, int B, int N, int K, int d, float *sums, float *first,
+             cudaStream_t s) {
   static bool attr = false;
   const int shm = kWarps * 2 * kBufBytes;
   if (!attr) {
@@ -303,22 +301,22 @@ int launch16(const void *x, const int32_t *skeys, const int32_t *perm, int B, in
   const int colblocks = (d + 127) / 128;
   const long long items = (long long)B * pieces * colblocks;
   const unsigned grid = (unsigned)((items + kWarps - 1) / kWarps);
-  k_segreduce16<T><<<grid, kWarps * 32, shm, s>>>((const T *)x, skeys, perm, N, K, d, pieces, colblocks,
-                                                  items, sums, first);
+  k_segreduce16<T><<<grid, kWarps * 32, shm, s>>>((const T *)x, kv, N, K, d, pieces, colblocks, items,
+                                                  sums, first);
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
 
 template <typename T, int VEC>
-int launch(const void *x, const int32_t *skeys, const int32_t *perm, int B, int N, int K, int d,
-           float *sums, float *first, cudaStream_t s) {
+int launch(const void *x, const int2 *kv, int B, int N, int K, int d, float *sums, float *first,
+           cudaStream_t s) {
   const int pieces = (N + kPiece - 1) / kPiece;
   const int colblocks = (d + 32 * VEC - 1) / (32 * VEC);
   const long long items = (long long)B * pieces * colblocks;
   const unsigned grid = (unsigned)((items + kWarps - 1) / kWarps);
-  k_segreduce<T, VEC><<<grid, kWarps * 32, 0, s>>>((const T *)x, skeys, perm, N, K, d, pieces,
-                                                   colblocks, items, sums, first);
+  k_segreduce<T, VEC><<<grid, kWarps * 32, 0, s>>>((const T *)x, kv, N, K, d, pieces, colblocks,
+                                                   items, sums, first);
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;
@@ -326,12 +324,12 @@ int launch(const void *x, const int32_t *skeys, const int32_t *perm, int B, int 
 
 }  // namespace
 
-int launch_segreduce(const void *x, int dtype, const int32_t *skeys, const int32_t *perm, int B,
-                     long long N, int K, int d, float *sums, float *first, cudaStream_t s) {
-  if (dtype == FK_F16) return launch16<__half>(x, skeys, perm, B, (int)N, K, d, sums, first, s);
-  if (dtype == FK_BF16) return launch16<__nv_bfloat16>(x, skeys, perm, B, (int)N, K, d, sums, first, s);
-  if (d % 4 == 0) return launch<float, 4>(x, skeys, perm, B, (int)N, K, d, sums, first, s);
-  return launch<float, 1>(x, skeys, perm, B, (int)N, K, d, sums, first, s);
+int launch_segreduce(const void *x, int dtype, const int2 *kv, int B, long long N, int K, int d,
+                     float *sums, float *first, cudaStream_t s) {
+  if (dtype == FK_F16) return launch16<__half>(x, kv, B, (int)N, K, d, sums, first, s);
+  if (dtype == FK_BF16) return launch16<__nv_bfloat16>(x, kv, B, (int)N, K, d, sums, first, s);
+  if (d % 4 == 0) return launch<float, 4>(x, kv, B, (int)N, K, d, sums, first, s);
+  return launch<float, 1>(x, kv, B, (int)N, K, d, sums, first, s);
 }
 
 }  // namespace fk

@@ -16,10 +16,12 @@
 //   k_scan_tiles   per (32 bins, batch): the exclusive prefix over tiles of
 //                  every bin, in place, and the bin totals -> counts,
 //   k_tile_scatter block scan of the counts -> bin offsets (written once per
-//                  batch); per-warp counts again, their prefix over the 8
-//                  warps on top of offsets[bin] + H[tile][bin], then every
-//                  warp ranks its rounds in order: equal digits inside a round
-//                  are ranked with a per-bit ballot mask.
+//                  batch) plus H[tile][bin] -> the tile's bases; per-warp
+//                  counts again, their prefix over the 8 warps on top of the
+//                  bases, then every warp ranks its rounds in order: equal
+//                  digits inside a round are ranked with a per-bit ballot
+//                  mask.  The update takes the sorted (id, point) pairs as one
+//                  8-byte store per point.
 // Stability: tiles are ordered by the tile prefix, warps inside a tile by the
 // warp prefix, points of a warp by the in-order rounds and the lane rank.
 #include "fk_internal.h"
@@ -74,20 +76,30 @@ struct WarpKeys {
   unsigned peers[kRounds];
 };
 
-__device__ __forceinline__ void load_warp_keys(WarpKeys &wk, const int32_t *kb, long long base,
-                                               int N, const PassCfg &pc, int K, int *err,
-                                               int lane) {
+__device__ __forceinline__ void fetch_warp_keys(WarpKeys &wk, const int32_t *kb, long long base,
+                                                int N, int lane) {
 #pragma unroll
   for (int r = 0; r < kRounds; ++r) {
     const long long i = base + r * 32 + lane;
     wk.key[r] = i < N ? __ldg(kb + i) : 0;
   }
+}
+
+__device__ __forceinline__ void rank_warp_keys(WarpKeys &wk, long long base, int N,
+                                               const PassCfg &pc, int K, int *err, int lane) {
 #pragma unroll
   for (int r = 0; r < kRounds; ++r) {
     const long long i = base + r * 32 + lane;
     wk.dg[r] = digit_of(wk.key[r], i < N, pc, K, err);
     wk.peers[r] = peers_of(wk.dg[r], pc.nbits);
   }
+}
+
+__device__ __forceinline__ void load_warp_keys(WarpKeys &wk, const int32_t *kb, long long base,
+                                               int N, const PassCfg &pc, int K, int *err,
+                                               int lane) {
+  fetch_warp_keys(wk, kb, base, N, lane);
+  rank_warp_keys(wk, base, N, pc, K, err, lane);
 }
 
 // cnt[dg] += number of this warp's points with digit dg (one leader per round
@@ -101,15 +113,22 @@ __device__ __forceinline__ void count_warp(uint32_t *cnt, const WarpKeys &wk, in
   }
 }
 
-// out[bin] = sum of counts[bin'] over bin' < bin, for bins <= kSortThreads * 16
-// (a block-wide exclusive scan; every thread of the CTA calls it).
-__device__ __forceinline__ void block_excl_scan(const int32_t *counts, int bins, uint32_t *out) {
+// out[bin] = gb[bin] + sum of counts[bin'] over bin' < bin, for bins <=
+// kSortThreads * 16: the first sorted position of the tile's points with this
+// digit (a block-wide exclusive scan; every thread of the CTA calls it).  The
+// counts and the tile prefixes gb are fetched in one pass, so their latencies
+// overlap.
+__device__ __forceinline__ void tile_bases(const int32_t *counts, const uint32_t *gb, int bins,
+                                           uint32_t *out) {
   __shared__ uint32_t wsum[kSortWarps];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int per = (bins + kSortThreads - 1) / kSortThreads;
   const int lo = min(bins, t * per), hi = min(bins, lo + per);
   uint32_t local = 0;
-  for (int bin = lo; bin < hi; ++bin) local += (uint32_t)counts[bin];
+  for (int bin = lo; bin < hi; ++bin) {
+    local += (uint32_t)__ldg(counts + bin);
+    out[bin] = __ldg(gb + bin);
+  }
   uint32_t incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -131,8 +150,8 @@ __device__ __forceinline__ void block_excl_scan(const int32_t *counts, int bins,
   __syncthreads();
   uint32_t run = wsum[warp] + incl - local;
   for (int bin = lo; bin < hi; ++bin) {
-    out[bin] = run;
-    run += (uint32_t)counts[bin];
+    out[bin] += run;
+    run += (uint32_t)__ldg(counts + bin);
   }
   __syncthreads();
 }
@@ -199,29 +218,28 @@ __global__ void __launch_bounds__(kSortThreads) k_scan_tiles(uint32_t *__restric
   }
 }
 
-// Stable scatter: vals_out[pos] = vals_in ? vals_in[i] : i and keys_out[pos] = key,
+// Stable scatter of tile `tile`: the point at position i goes to
 // pos = offsets[digit] + G[tile][digit] + (earlier warps of the tile with the
 // digit) + rank of the point among the warp's earlier points with the digit.
-// The CTA of tile 0 also writes offsets_out[b] (when not NULL).
+// It writes vals_out[pos] = vals_in ? vals_in[i] : i and keys_out[pos] = key
+// (each when not NULL), or the pair kv_out[pos] = (key, value): one 8-byte
+// store per point where the update needs both.  The CTA of tile 0 also writes
+// offsets_out[b] (when not NULL).
 __global__ void __launch_bounds__(kSortThreads) k_tile_scatter(
     const int32_t *__restrict__ keys, const int32_t *__restrict__ vals_in, int N, int K, int T,
     PassCfg pc, const uint32_t *__restrict__ G, const int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets_out, int32_t *__restrict__ keys_out,
-    int32_t *__restrict__ vals_out, int *err) {
-  extern __shared__ uint32_t sm[];  // off[bins], cnt[kSortWarps][bins]
+    int32_t *__restrict__ vals_out, int2 *__restrict__ kv_out, int *err) {
+  extern __shared__ uint32_t sm[];  // base[bins], cnt[kSortWarps][bins]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, b = blockIdx.y;
   const int bins = pc.bins;
-  uint32_t *off = sm;
+  uint32_t *tb = sm;
   uint32_t *cnt_all = sm + bins;
-  for (int e = threadIdx.x; e < kSortWarps * bins; e += kSortThreads) cnt_all[e] = 0;
-  block_excl_scan(counts + (size_t)b * bins, bins, off);  // ends with __syncthreads
-  if (tile == 0 && offsets_out)
-    for (int bin = threadIdx.x; bin < bins; bin += kSortThreads)
-      offsets_out[(size_t)b * bins + bin] = (int32_t)off[bin];
   const long long base = (long long)tile * kSortTile + warp * kWarpPoints;
+  // the keys (and values) are fetched first; their latency overlaps the scan
   WarpKeys wk;
-  load_warp_keys(wk, keys + (size_t)b * N, base, N, pc, K, err, lane);
+  fetch_warp_keys(wk, keys + (size_t)b * N, base, N, lane);
   int vals[kRounds];
   if (vals_in) {
 #pragma unroll
@@ -230,12 +248,17 @@ __global__ void __launch_bounds__(kSortThreads) k_tile_scatter(
       vals[r] = i < N ? __ldg(vals_in + (size_t)b * N + i) : 0;
     }
   }
+  for (int e = threadIdx.x; e < kSortWarps * bins; e += kSortThreads) cnt_all[e] = 0;
+  tile_bases(counts + (size_t)b * bins, G + ((size_t)b * T + tile) * bins, bins, tb);
+  if (tile == 0 && offsets_out)  // tile 0's prefix is zero: its bases are the offsets
+    for (int bin = threadIdx.x; bin < bins; bin += kSortThreads)
+      offsets_out[(size_t)b * bins + bin] = (int32_t)tb[bin];
+  rank_warp_keys(wk, base, N, pc, K, err, lane);
   uint32_t *cnt = cnt_all + warp * bins;
   count_warp(cnt, wk, lane);
   __syncthreads();
-  const uint32_t *gb = G + ((size_t)b * T + tile) * bins;
   for (int bin = threadIdx.x; bin < bins; bin += kSortThreads) {
-    uint32_t run = off[bin] + gb[bin];
+    uint32_t run = tb[bin];
 #pragma unroll
     for (int w = 0; w < kSortWarps; ++w) {
       const uint32_t v = cnt_all[w * bins + bin];
@@ -245,7 +268,8 @@ __global__ void __launch_bounds__(kSortThreads) k_tile_scatter(
   }
   __syncthreads();
   int32_t *ko = keys_out ? keys_out + (size_t)b * N : nullptr;
-  int32_t *vo = vals_out + (size_t)b * N;
+  int32_t *vo = vals_out ? vals_out + (size_t)b * N : nullptr;
+  int2 *kvo = kv_out ? kv_out + (size_t)b * N : nullptr;
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
   for (int r = 0; r < kRounds; ++r) {
@@ -255,7 +279,9 @@ __global__ void __launch_bounds__(kSortThreads) k_tile_scatter(
     __syncwarp();
     if (dg != kNoDigit) {
       if (lane == __ffs(peers) - 1) cnt[dg] += __popc(peers);
-      vo[pos] = vals_in ? vals[r] : (int32_t)(base + r * 32 + lane);
+      const int32_t val = vals_in ? vals[r] : (int32_t)(base + r * 32 + lane);
+      if (kvo) kvo[pos] = make_int2(wk.key[r], val);
+      if (vo) vo[pos] = val;
       if (ko) ko[pos] = wk.key[r];
     }
     __syncwarp();
@@ -345,7 +371,7 @@ int set_attrs() {
 // offsets_out (B, bins), when not NULL, their exclusive scan.
 int one_pass(Workspace *ws, const int32_t *keys_in, const int32_t *vals_in, int B, int N, int K,
              int T, PassCfg pc, int32_t *digit_counts, int32_t *offsets_out, int32_t *keys_out,
-             int32_t *vals_out, cudaStream_t s, bool have_hist = false) {
+             int32_t *vals_out, int2 *kv_out, cudaStream_t s, bool have_hist = false) {
   FK_TRY(ensure(ws->table, (size_t)B * T * pc.bins * sizeof(uint32_t)));
   uint32_t *H = (uint32_t *)ws->table.p;
   const dim3 grid((unsigned)T, (unsigned)B);
@@ -361,7 +387,8 @@ int one_pass(Workspace *ws, const int32_t *keys_in, const int32_t *vals_in, int 
   count_launch();
   FK_CUDA(cudaGetLastError());
   k_tile_scatter<<<grid, kSortThreads, shm_s, s>>>(keys_in, vals_in, N, K, T, pc, H, digit_counts,
-                                                   offsets_out, keys_out, vals_out, ws->err);
+                                                   offsets_out, keys_out, vals_out, kv_out,
+                                                   ws->err);
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;
@@ -376,7 +403,7 @@ size_t sort_table_bytes(int B, long long N, int K) {
 }
 
 int run_sort_prehist(Workspace *ws, const int32_t *ids, int B, long long N_, int K, int32_t *counts,
-                     int32_t *offsets, int32_t *perm, int32_t *keys_out, cudaStream_t s) {
+                     int32_t *offsets, int32_t *perm, int2 *kv_out, cudaStream_t s) {
   if (!sort_single_pass(K)) return set_error(FK_EUNSUPPORTED, "fused histogram needs K <= 4096");
   FK_TRY(set_attrs());
   const int N = (int)N_;
@@ -391,11 +418,11 @@ int run_sort_prehist(Workspace *ws, const int32_t *ids, int B, long long N_, int
     off = (int32_t *)ws->offsets.p;
   }
   PassCfg pc{0, 0xffffffffu, K, bits_for(K), true};
-  return one_pass(ws, ids, nullptr, B, N, K, T, pc, cnt, off, keys_out, perm, s, true);
+  return one_pass(ws, ids, nullptr, B, N, K, T, pc, cnt, off, nullptr, perm, kv_out, s, true);
 }
 
 int run_sort(Workspace *ws, const int32_t *ids, int B, long long N_, int K, int32_t *counts,
-             int32_t *offsets, int32_t *perm, int32_t *keys_out, cudaStream_t s) {
+             int32_t *offsets, int32_t *perm, int2 *kv_out, cudaStream_t s) {
   FK_TRY(set_attrs());
   const int N = (int)N_;
   const int T = (int)((N_ + kSortTile - 1) / kSortTile);
@@ -412,7 +439,7 @@ int run_sort(Workspace *ws, const int32_t *ids, int B, long long N_, int K, int3
       off = (int32_t *)ws->offsets.p;
     }
     PassCfg pc{0, 0xffffffffu, K, nbits, true};
-    return one_pass(ws, ids, nullptr, B, N, K, T, pc, cnt, off, keys_out, perm, s);
+    return one_pass(ws, ids, nullptr, B, N, K, T, pc, cnt, off, nullptr, perm, kv_out, s);
   }
   const int lo = (nbits + 1) / 2, hi = nbits - lo;
   const size_t nb = (size_t)B * N * sizeof(int32_t);
@@ -423,9 +450,9 @@ int run_sort(Workspace *ws, const int32_t *ids, int B, long long N_, int K, int3
   FK_TRY(ensure(ws->digit_off, (size_t)B * (1 << kMaxDigitBits) * sizeof(int32_t)));
   int32_t *dcnt = (int32_t *)ws->digit_off.p;
   PassCfg p1{0, (1u << lo) - 1u, 1 << lo, lo, true};
-  FK_TRY(one_pass(ws, ids, nullptr, B, N, K, T, p1, dcnt, nullptr, kt, vt, s));
+  FK_TRY(one_pass(ws, ids, nullptr, B, N, K, T, p1, dcnt, nullptr, kt, vt, nullptr, s));
   PassCfg p2{lo, (1u << hi) - 1u, 1 << hi, hi, false};
-  FK_TRY(one_pass(ws, kt, vt, B, N, K, T, p2, dcnt, nullptr, keys_out, perm, s));
+  FK_TRY(one_pass(ws, kt, vt, B, N, K, T, p2, dcnt, nullptr, nullptr, perm, kv_out, s));
   // cluster counts and offsets (a pass's digit totals are not cluster totals)
   FK_CUDA(cudaMemsetAsync(cnt, 0, (size_t)B * K * sizeof(int32_t), s));
   const int use_smem = (size_t)K * 4 <= 64 * 1024 ? 1 : 0;
