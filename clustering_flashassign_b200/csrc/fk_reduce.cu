@@ -170,18 +170,35 @@ __device__ __forceinline__ void issue_batch(uint32_t dst, const T *xb, int d, in
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-template <typename T>
-__device__ __forceinline__ void add_row(float (&acc)[4], const uint8_t *slice) {
+// acc[c] += element c of the row slice (4 consecutive 16-bit elements): the
+// mixed-precision add widens the 16-bit operand exactly and rounds the fp32
+// sum once, so it equals a conversion followed by an fp32 add, in one
+// instruction instead of two.
+template <typename T> __device__ __forceinline__ void add_row(float (&acc)[4], const uint8_t *slice);
+template <> __device__ __forceinline__ void add_row<__half>(float (&acc)[4], const uint8_t *slice) {
   const uint2 u = *reinterpret_cast<const uint2 *>(slice);
-  float2 f0, f1;
-  if constexpr (std::is_same<T, __half>::value) {
-    f0 = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
-    f1 = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
-  } else {
-    f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-    f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-  }
-  acc[0] += f0.x; acc[1] += f0.y; acc[2] += f1.x; acc[3] += f1.y;
+  asm("{\n\t.reg .f16 a0, a1, a2, a3;\n\t"
+      "mov.b32 {a0, a1}, %4;\n\t"
+      "mov.b32 {a2, a3}, %5;\n\t"
+      "add.rn.f32.f16 %0, a0, %0;\n\t"
+      "add.rn.f32.f16 %1, a1, %1;\n\t"
+      "add.rn.f32.f16 %2, a2, %2;\n\t"
+      "add.rn.f32.f16 %3, a3, %3;\n\t}"
+      : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+      : "r"(u.x), "r"(u.y));
+}
+template <>
+__device__ __forceinline__ void add_row<__nv_bfloat16>(float (&acc)[4], const uint8_t *slice) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(slice);
+  asm("{\n\t.reg .b16 a0, a1, a2, a3;\n\t"
+      "mov.b32 {a0, a1}, %4;\n\t"
+      "mov.b32 {a2, a3}, %5;\n\t"
+      "add.rn.f32.bf16 %0, a0, %0;\n\t"
+      "add.rn.f32.bf16 %1, a1, %1;\n\t"
+      "add.rn.f32.bf16 %2, a2, %2;\n\t"
+      "add.rn.f32.bf16 %3, a3, %3;\n\t}"
+      : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+      : "r"(u.x), "r"(u.y));
 }
 
 template <typename T>
@@ -263,17 +280,16 @@ __global__ void __launch_bounds__(kWarps * 32) k_segreduce16(const T *__restrict
         start = j0 + 32 * kc + q;
       }
       if (key >= 0 && active) {
+        // even rows of the run into acc, odd rows into a2 (two short chains)
+        float a2[4] = {0.f, 0.f, 0.f, 0.f};
         int r = q;
-        for (; r + 4 <= e; r += 4) {
-          float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
-          add_row<T>(s, slab + (r - q0) * kSliceBytes);
-          add_row<T>(s2, slab + (r + 1 - q0) * kSliceBytes);
-          add_row<T>(s, slab + (r + 2 - q0) * kSliceBytes);
-          add_row<T>(s2, slab + (r + 3 - q0) * kSliceBytes);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[c] += s[c] + s2[c];
+        for (; r + 2 <= e; r += 2) {
+          add_row<T>(acc, slab + (r - q0) * kSliceBytes);
+          add_row<T>(a2, slab + (r + 1 - q0) * kSliceBytes);
         }
-        for (; r < e; ++r) add_row<T>(acc, slab + (r - q0) * kSliceBytes);
+        if (r < e) add_row<T>(acc, slab + (r - q0) * kSliceBytes);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[c] += a2[c];
       }
       q = e;
     }
