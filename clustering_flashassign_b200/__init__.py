@@ -10,6 +10,14 @@ fallback: when libfk.so is missing, importing this package raises.
     fk_update(x, ids, centers, counts=None)     sort-inverse update, centers (B,K,d) fp32 in/out
     fk_sort(ids, K, perm, counts=None, offsets=None)
     fk_lloyd(x, init_centers, max_iter, tol, ids, centers) -> iterations run
+
+Per-rank pieces of a data-parallel run (points of a batch split over ranks;
+the loop that joins them with an all-reduce is clustering_flashassign_b200.dist):
+
+    fk_point_norms(x, xn)                       ||x_i||^2 for the tensor-core assign
+    fk_init_centers(init, centers)              fp32 master copy of the initial centroids
+    fk_lloyd_step_partial(x, xn, centers_dt, ids, sums, counts)   assign + unnormalised update
+    fk_update_finalize(sums, counts, centers, centers_dt, max_shift)
 """
 from __future__ import annotations
 
@@ -29,7 +37,8 @@ DTYPES = {torch.float32: FK_F32, torch.float16: FK_F16, torch.bfloat16: FK_BF16}
 
 EXPORTS = ["fk_assign", "fk_update", "fk_sort", "fk_lloyd", "fk_assign_noalloc", "fk_status_string",
            "fk_last_error", "fk_device_error", "fk_release", "fk_profile_enable", "fk_profile_read",
-           "fk_launch_count", "fk_version", "fk_selftest_bounded_wait"]
+           "fk_launch_count", "fk_version", "fk_selftest_bounded_wait", "fk_point_norms",
+           "fk_init_centers", "fk_lloyd_step_partial", "fk_update_finalize"]
 
 
 class FkError(RuntimeError):
@@ -76,6 +85,11 @@ def _load():
         "fk_launch_count": (LL, []),
         "fk_version": (I, []),
         "fk_selftest_bounded_wait": (I, [LL, P]),
+        "fk_point_norms": (I, [P, I, LL, I, I, P, P]),
+        "fk_init_centers": (I, [P, I, I, I, I, P, P]),
+        "fk_lloyd_step_partial": (I, [ctypes.POINTER(FkShape), P, P, P, P, P, P, P,
+                                      ctypes.POINTER(FkOptions)]),
+        "fk_update_finalize": (I, [P, P, I, I, I, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -165,6 +179,46 @@ def fk_lloyd(x: torch.Tensor, init_centers: torch.Tensor, max_iter: int, tol: fl
                         _ptr(ids), _ptr(centers), _stream(stream), ctypes.byref(iters),
                         ctypes.byref(opts)), "fk_lloyd")
     return iters.value
+
+
+def fk_point_norms(x: torch.Tensor, xn: torch.Tensor, stream=None) -> torch.Tensor:
+    """xn (B, N) fp32 = ||x[b, i]||^2 of fp16 / bf16 points (B, N, d)."""
+    B, N, d = x.shape
+    _check(lib.fk_point_norms(_ptr(x), B, N, d, _dtype_code(x), _ptr(xn), _stream(stream)),
+           "fk_point_norms")
+    return xn
+
+
+def fk_init_centers(init: torch.Tensor, centers: torch.Tensor, stream=None) -> torch.Tensor:
+    """centers (B, K, d) fp32 = init (B, K, d) in the points' dtype, widened exactly."""
+    B, K, d = init.shape
+    _check(lib.fk_init_centers(_ptr(init), B, K, d, _dtype_code(init), _ptr(centers), _stream(stream)),
+           "fk_init_centers")
+    return centers
+
+
+def fk_lloyd_step_partial(x: torch.Tensor, xn, centers_dt: torch.Tensor, ids: torch.Tensor,
+                          sums: torch.Tensor, counts: torch.Tensor, stream=None,
+                          chunk_points: int = 0) -> None:
+    """Assign this block of points (device or pinned host) and write its per-cluster
+    sums (B, K, d) fp32 and counts (B, K) int32 (no division)."""
+    B, N, d = x.shape
+    K = centers_dt.shape[1]
+    shape = FkShape(B, N, K, d, _dtype_code(x))
+    opts = FkOptions(FK_HOST_AUTO, chunk_points, 0)
+    _check(lib.fk_lloyd_step_partial(ctypes.byref(shape), _ptr(x), _ptr(xn), _ptr(centers_dt), _ptr(ids),
+                                     _ptr(sums), _ptr(counts), _stream(stream), ctypes.byref(opts)),
+           "fk_lloyd_step_partial")
+
+
+def fk_update_finalize(sums: torch.Tensor, counts: torch.Tensor, centers: torch.Tensor,
+                       centers_dt=None, max_shift=None, dtype=None, stream=None) -> torch.Tensor:
+    """centers = sums / counts where counts > 0 (else unchanged); centers_dt = rounded copy."""
+    B, K, d = centers.shape
+    code = _dtype_code(centers_dt) if centers_dt is not None else DTYPES[dtype or torch.float32]
+    _check(lib.fk_update_finalize(_ptr(sums), _ptr(counts), B, K, d, code, _ptr(centers), _ptr(centers_dt),
+                                  _ptr(max_shift), _stream(stream)), "fk_update_finalize")
+    return centers
 
 
 def fk_device_error(stream=None) -> int:

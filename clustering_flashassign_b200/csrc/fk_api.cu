@@ -124,26 +124,82 @@ int ensure_copy_engine(Workspace *ws) {
   return FK_OK;
 }
 
-// Out-of-core Lloyd: x stays in host memory and is re-streamed every iteration
-// in chunks, double-buffered so the copy of chunk j+1 overlaps the compute of
-// chunk j ("flash-kmeans and the return of exact K-Means on the GPU", section
-// "Multi-GPU scaling without a NCCL dependency": per-device double-buffered
-// host-to-device plus compute pipeline, and the next iteration's first block
-// prefetched while the current iteration reduces).  Assign, sort and segment
-// reduce run per chunk; counts and sums accumulate over the chunks and the
-// finalize runs once per iteration.
-int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void *init_dev,
-                   int max_iter, float tol, int32_t *ids_dev, float *cen_dev, cudaStream_t s,
-                   int *iters_run, long long chunk, int verbose) {
+// Scratch of the streamed pipeline: the copy stream and events, two chunk
+// buffers, and the per-chunk update scratch (one batch of `chunk` points).
+int prepare_streamed(Workspace *ws, const fk_shape &sh, long long chunk) {
+  FK_TRY(ensure_copy_engine(ws));
+  for (int i = 0; i < 2; ++i) FK_TRY(ensure(ws->chunk[i], (size_t)chunk * sh.d * esize(sh.dtype)));
+  FK_TRY(ensure(ws->counts, (size_t)sh.K * sizeof(int32_t)));
+  return prepare_update(ws, 1, chunk, sh.K, sh.d);
+}
+
+// One pass of the out-of-core pipeline over every batch: x stays in host
+// memory and is streamed in chunks, double-buffered so the copy of chunk j+1
+// overlaps the compute of chunk j ("flash-kmeans and the return of exact
+// K-Means on the GPU", section "Multi-GPU scaling without a NCCL dependency":
+// per-device double-buffered host-to-device plus compute pipeline).  Each
+// chunk is assigned against `cassign` (B, K, d) in x's dtype, sorted and
+// segment-reduced, and its sums and counts are folded into gsum / gcounts
+// (zeroed first).  ws->stream_job numbers the chunks across passes, so the
+// two buffers keep alternating and the next pass's first copy can start while
+// the current pass is still being reduced.
+int streamed_pass(Workspace *ws, const fk_shape &sh, const char *xh, long long chunk,
+                  const void *cassign, const char *cnx, int32_t *ids_dev, float *gsum,
+                  int32_t *gcounts, cudaStream_t s) {
   const int B = sh.B, K = sh.K, d = sh.d, dtype = sh.dtype;
   const long long N = sh.N;
   const size_t es = esize(dtype);
   const long long Kpad = kpad_of(K);
-  if (chunk <= 0) chunk = 1LL << 24;
-  if (chunk > N) chunk = N;
   const long long per_b = (N + chunk - 1) / chunk;
-  FK_TRY(ensure_copy_engine(ws));
-  for (int i = 0; i < 2; ++i) FK_TRY(ensure(ws->chunk[i], (size_t)chunk * d * es));
+  int32_t *counts = (int32_t *)ws->counts.p;
+  float *sums = (float *)ws->sums.p, *first = (float *)ws->first.p;
+  int2 *kv = (int2 *)ws->kv.p;
+  int32_t *offsets = (int32_t *)ws->offsets.p;
+  note_update_call();
+  FK_CUDA(cudaMemsetAsync(gcounts, 0, (size_t)B * K * sizeof(int32_t), s));
+  FK_CUDA(cudaMemsetAsync(gsum, 0, (size_t)B * K * d * sizeof(float), s));
+  for (int b = 0; b < B; ++b) {
+    for (long long ci = 0; ci < per_b; ++ci, ++ws->stream_job) {
+      const int buf = (int)(ws->stream_job & 1);
+      const long long n0 = ci * chunk;
+      const long long nc = (n0 + chunk <= N) ? chunk : N - n0;
+      void *xb = ws->chunk[buf].p;
+      FK_CUDA(cudaStreamWaitEvent(ws->copy_stream, ws->freed[buf], 0));
+      FK_CUDA(cudaMemcpyAsync(xb, xh + ((size_t)b * N + n0) * d * es, (size_t)nc * d * es,
+                              cudaMemcpyHostToDevice, ws->copy_stream));
+      FK_CUDA(cudaEventRecord(ws->ready[buf], ws->copy_stream));
+      FK_CUDA(cudaStreamWaitEvent(s, ws->ready[buf], 0));
+      int32_t *idc = ids_dev + (size_t)b * N + n0;
+      const void *cb = (const char *)cassign + (size_t)b * K * d * es;
+      FK_TRY(do_assign_resident(ws, xb, cb, cnx ? cnx + ext_bytes(b, Kpad) : nullptr, nullptr, 1, nc, K,
+                                d, dtype, Kpad, idc, s));
+      {
+        PhaseTimer t(PH_SORT, s);
+        FK_TRY(run_sort(ws, idc, 1, nc, K, counts, offsets, nullptr, kv, s));
+      }
+      {
+        PhaseTimer t(PH_REDUCE, s);
+        FK_TRY(launch_segreduce(xb, dtype, kv, 1, nc, K, d, sums, first, s));
+        FK_TRY(launch_accumulate(sums, first, pieces_of(nc), counts, offsets, 1, K, d,
+                                 gsum + (size_t)b * K * d, gcounts + (size_t)b * K, false, s));
+      }
+      FK_CUDA(cudaEventRecord(ws->freed[buf], s));
+    }
+  }
+  return FK_OK;
+}
+
+// Out-of-core Lloyd: one streamed pass per iteration (assign, sort and
+// segment reduce per chunk), then one finalize per iteration.
+int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void *init_dev,
+                   int max_iter, float tol, int32_t *ids_dev, float *cen_dev, cudaStream_t s,
+                   int *iters_run, long long chunk, int verbose) {
+  const int B = sh.B, K = sh.K, d = sh.d, dtype = sh.dtype;
+  const size_t es = esize(dtype);
+  const long long Kpad = kpad_of(K);
+  if (chunk <= 0) chunk = 1LL << 24;
+  if (chunk > sh.N) chunk = sh.N;
+  FK_TRY(prepare_streamed(ws, sh, chunk));
   void *ch = nullptr;
   char *cnx = nullptr;
   if (dtype != FK_F32) {
@@ -152,54 +208,17 @@ int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void
     ch = ws->ch.p;
     cnx = (char *)ws->cn.p;
   }
-  // per chunk: counts, offsets, owner / continuation partials (one batch);
   // per iteration: running sums and counts of every batch
-  FK_TRY(ensure(ws->counts, (size_t)K * sizeof(int32_t)));
   FK_TRY(ensure(ws->gsum, (size_t)B * K * d * sizeof(float)));
   FK_TRY(ensure(ws->gcounts, (size_t)B * K * sizeof(int32_t)));
-  int32_t *counts = (int32_t *)ws->counts.p, *gcounts = (int32_t *)ws->gcounts.p;
+  int32_t *gcounts = (int32_t *)ws->gcounts.p;
   float *gsum = (float *)ws->gsum.p;
   FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cnx, ws->err, s));
-  FK_TRY(prepare_update(ws, 1, chunk, K, d));
-  float *sums = (float *)ws->sums.p, *first = (float *)ws->first.p;
-  int2 *kv = (int2 *)ws->kv.p;
-  int32_t *offsets = (int32_t *)ws->offsets.p;
-  long long job = 0;
+  const void *cassign = dtype == FK_F32 ? (const void *)cen_dev : ch;
   int it = 0;
   for (it = 0; it < max_iter; ++it) {
-    note_update_call();
-    FK_CUDA(cudaMemsetAsync(gcounts, 0, (size_t)B * K * sizeof(int32_t), s));
-    FK_CUDA(cudaMemsetAsync(gsum, 0, (size_t)B * K * d * sizeof(float), s));
     FK_CUDA(cudaMemsetAsync(ws->maxshift, 0, sizeof(unsigned), s));
-    for (int b = 0; b < B; ++b) {
-      for (long long ci = 0; ci < per_b; ++ci, ++job) {
-        const int buf = (int)(job & 1);
-        const long long n0 = ci * chunk;
-        const long long nc = (n0 + chunk <= N) ? chunk : N - n0;
-        void *xb = ws->chunk[buf].p;
-        FK_CUDA(cudaStreamWaitEvent(ws->copy_stream, ws->freed[buf], 0));
-        FK_CUDA(cudaMemcpyAsync(xb, xh + ((size_t)b * N + n0) * d * es, (size_t)nc * d * es,
-                                cudaMemcpyHostToDevice, ws->copy_stream));
-        FK_CUDA(cudaEventRecord(ws->ready[buf], ws->copy_stream));
-        FK_CUDA(cudaStreamWaitEvent(s, ws->ready[buf], 0));
-        int32_t *idc = ids_dev + (size_t)b * N + n0;
-        const void *cb = dtype == FK_F32 ? (const void *)(cen_dev + (size_t)b * K * d)
-                                         : (const void *)((const char *)ch + (size_t)b * K * d * es);
-        FK_TRY(do_assign_resident(ws, xb, cb, cnx ? cnx + ext_bytes(b, Kpad) : nullptr, nullptr, 1, nc, K, d, dtype,
-                                  Kpad, idc, s));
-        {
-          PhaseTimer t(PH_SORT, s);
-          FK_TRY(run_sort(ws, idc, 1, nc, K, counts, offsets, nullptr, kv, s));
-        }
-        {
-          PhaseTimer t(PH_REDUCE, s);
-          FK_TRY(launch_segreduce(xb, dtype, kv, 1, nc, K, d, sums, first, s));
-          FK_TRY(launch_accumulate(sums, first, pieces_of(nc), counts, offsets, K, d,
-                                   gsum + (size_t)b * K * d, gcounts + (size_t)b * K, s));
-        }
-        FK_CUDA(cudaEventRecord(ws->freed[buf], s));
-      }
-    }
+    FK_TRY(streamed_pass(ws, sh, xh, chunk, cassign, cnx, ids_dev, gsum, gcounts, s));
     {
       PhaseTimer t(PH_FINALIZE, s);
       FK_TRY(launch_finalize(gsum, nullptr, 0, gcounts, nullptr, cen_dev, ch, cnx, dtype, B, K, d,
@@ -217,6 +236,32 @@ int lloyd_streamed(Workspace *ws, const fk_shape &sh, const char *xh, const void
   }
   *iters_run = it;
   return FK_OK;
+}
+
+// Steps a2-a5 without the division, on device-resident points: the
+// per-cluster sums (B, K, d) fp32 and counts (B, K) of these points, written
+// to the caller's buffers (an empty cluster gets zeros).  have_hist as in
+// do_update.
+int do_partial(Workspace *ws, const void *x, const int32_t *ids, int B, long long N, int K, int d,
+               int dtype, float *sums_out, int32_t *counts_out, cudaStream_t s, bool have_hist) {
+  note_update_call();
+  PhaseTimer whole(PH_UPDATE, s);
+  FK_TRY(prepare_update(ws, B, N, K, d));
+  int2 *kv = (int2 *)ws->kv.p;
+  int32_t *offsets = (int32_t *)ws->offsets.p;
+  float *sums = (float *)ws->sums.p, *first = (float *)ws->first.p;
+  {
+    PhaseTimer t(PH_SORT, s);
+    if (have_hist) FK_TRY(run_sort_prehist(ws, ids, B, N, K, counts_out, offsets, nullptr, kv, s));
+    else FK_TRY(run_sort(ws, ids, B, N, K, counts_out, offsets, nullptr, kv, s));
+  }
+  {
+    PhaseTimer t(PH_REDUCE, s);
+    FK_TRY(launch_segreduce(x, dtype, kv, B, N, K, d, sums, first, s));
+  }
+  PhaseTimer t(PH_FINALIZE, s);
+  return launch_accumulate(sums, first, pieces_of(N), counts_out, offsets, B, K, d, sums_out, nullptr,
+                           true, s);
 }
 
 }  // namespace
@@ -271,6 +316,94 @@ int fk_sort(const int32_t *ids, int B, long long N, int K, int32_t *counts, int3
   FK_TRY(workspace_for(s, &ws));
   PhaseTimer t(PH_SORT, s);
   return run_sort(ws, ids, B, N, K, counts, offsets, perm, nullptr, s);
+}
+
+int fk_point_norms(const void *x, int B, long long N, int d, int dtype, float *xn,
+                   fk_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FK_TRY(check_shape(B, N, 1, d, dtype));
+  if (dtype == FK_F32) return set_error(FK_EUNSUPPORTED, "point norms serve the fp16 / bf16 assign");
+  FK_TRY(check_ptr(x, "x", true));
+  FK_TRY(check_ptr(xn, "xn", false));
+  return launch_point_norms(x, dtype, (long long)B * N, d, xn, s);
+}
+
+int fk_init_centers(const void *init, int B, int K, int d, int dtype, float *centers,
+                    fk_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FK_TRY(check_shape(B, K, K, d, dtype));
+  FK_TRY(check_ptr(init, "init", false));
+  FK_TRY(check_ptr(centers, "centers", false));
+  Workspace *ws;
+  FK_TRY(workspace_for(s, &ws));
+  return launch_init_centers(init, dtype, B, K, d, kpad_of(K), centers, nullptr, nullptr, ws->err, s);
+}
+
+int fk_lloyd_step_partial(const fk_shape *shape, const void *x, const float *xn,
+                          const void *centers_dt, int32_t *ids, float *sums, int32_t *counts,
+                          fk_stream_t stream, const fk_options *opts) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!shape) return set_error(FK_EINVAL, "shape is NULL");
+  const fk_shape sh = *shape;
+  const int B = sh.B, K = sh.K, d = sh.d, dtype = sh.dtype;
+  const long long N = sh.N;
+  FK_TRY(check_shape(B, N, K, d, dtype));
+  const bool tc = dtype != FK_F32;
+  FK_TRY(check_ptr(x, "x", tc));
+  FK_TRY(check_ptr(centers_dt, "centers_dt", tc));
+  FK_TRY(check_ptr(ids, "ids", false));
+  FK_TRY(check_ptr(sums, "sums", false));
+  FK_TRY(check_ptr(counts, "counts", false));
+  const fk_options o = opts ? *opts : fk_options{FK_HOST_AUTO, 0, 0};
+  Workspace *ws;
+  FK_TRY(workspace_for(s, &ws));
+  const long long Kpad = kpad_of(K);
+  char *cnx = nullptr;
+  if (tc) {
+    FK_TRY(ensure(ws->cn, ext_bytes(B, Kpad)));
+    cnx = (char *)ws->cn.p;
+    FK_TRY(launch_prep_cn(centers_dt, dtype, B, K, d, Kpad, cnx, ws->err, s));
+  }
+  const Loc lx = locate(x);
+  if (lx == LOC_HOST_PAGEABLE) return set_error(FK_EINVAL, "x must be device or pinned host memory");
+  if (lx == LOC_HOST_PINNED) {
+    long long chunk = o.chunk_points > 0 ? o.chunk_points : (1LL << 24);
+    if (chunk > N) chunk = N;
+    FK_TRY(prepare_streamed(ws, sh, chunk));
+    return streamed_pass(ws, sh, (const char *)x, chunk, centers_dt, cnx, ids, sums, counts, s);
+  }
+  // With K <= 4096 the assign counts every id into the sort's tile histogram.
+  const bool fuse = tc && sort_single_pass(K);
+  uint32_t *hist = nullptr;
+  if (fuse) {
+    const size_t hist_bytes = sort_table_bytes(B, N, K);
+    FK_TRY(ensure(ws->table, hist_bytes));
+    hist = (uint32_t *)ws->table.p;
+    FK_CUDA(cudaMemsetAsync(hist, 0, hist_bytes, s));
+  }
+  const float *xnr = (tc && d <= 2 * kBlockK) ? xn : nullptr;
+  FK_TRY(do_assign_resident(ws, x, centers_dt, cnx, xnr, B, N, K, d, dtype, Kpad, ids, s, hist));
+  return do_partial(ws, x, ids, B, N, K, d, dtype, sums, counts, s, fuse);
+}
+
+int fk_update_finalize(const float *sums, const int32_t *counts, int B, int K, int d, int dtype,
+                       float *centers, void *centers_dt, float *max_shift, fk_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FK_TRY(check_shape(B, K, K, d, dtype));
+  FK_TRY(check_ptr(sums, "sums", false));
+  FK_TRY(check_ptr(counts, "counts", false));
+  FK_TRY(check_ptr(centers, "centers", true));
+  Workspace *ws;
+  FK_TRY(workspace_for(s, &ws));
+  FK_CUDA(cudaMemsetAsync(ws->maxshift, 0, sizeof(unsigned), s));
+  {
+    PhaseTimer t(PH_FINALIZE, s);
+    FK_TRY(launch_finalize(sums, nullptr, 0, counts, nullptr, centers, dtype == FK_F32 ? nullptr : centers_dt,
+                           nullptr, dtype, B, K, d, kpad_of(K), ws->maxshift, false, ws->err, s));
+  }
+  if (max_shift)
+    FK_CUDA(cudaMemcpyAsync(max_shift, ws->maxshift, sizeof(float), cudaMemcpyDeviceToDevice, s));
+  return FK_OK;
 }
 
 int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int max_iter,

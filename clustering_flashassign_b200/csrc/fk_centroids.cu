@@ -236,27 +236,43 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   }
 }
 
-// Streamed path: fold one chunk's segment sums and counts into the running
-// totals of its batch (chunks are folded in order, so the totals are
+// Per-cluster totals of the segment partials, grid (blocks, B).  overwrite:
+// gsum[b][k] = the cluster's sum (zero for an empty cluster), the counts are
+// already final; otherwise gsum[b][k] += it and gcounts[b][k] += counts[b][k]
+// (the streamed path folds its chunks in order, so the totals are
 // reproducible).
 template <bool V4>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     k_accumulate(const float *__restrict__ sums, const float *__restrict__ first, int pieces,
                  const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets, int K,
-                 int d, float *__restrict__ gsum, int32_t *__restrict__ gcounts) {
+                 int d, float *__restrict__ gsum, int32_t *__restrict__ gcounts, int overwrite) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  sums += (size_t)b * K * d;
+  first += (size_t)b * pieces * d;
+  counts += (size_t)b * K;
+  offsets += (size_t)b * K;
+  gsum += (size_t)b * K * d;
   for (long long k = (long long)blockIdx.x * kWarpsPerBlock + warp; k < K;
        k += (long long)gridDim.x * kWarpsPerBlock) {
     const int cnt = counts[k];
-    if (cnt == 0) continue;
+    const size_t w_off = (size_t)k * d;
+    if (cnt == 0) {
+      if (overwrite)
+        for_lane_elems<V4>(d, lane, [&](int j, int n) {
+          for (int e = 0; e < n; ++e) gsum[w_off + j + e] = 0.f;
+        });
+      continue;
+    }
     const int off = offsets[k];
     const int p0 = off / kPiece, pl = (off + cnt - 1) / kPiece;
-    const size_t w_off = (size_t)k * d;
     for_lane_elems<V4>(d, lane, [&](int j, int n) {
-      for (int e = 0; e < n; ++e)
-        gsum[w_off + j + e] += seg_sum<true>(sums, first, w_off, 0, d, p0, pl, j + e);
+      for (int e = 0; e < n; ++e) {
+        const float v = seg_sum<true>(sums, first, w_off, 0, d, p0, pl, j + e);
+        gsum[w_off + j + e] = overwrite ? v : gsum[w_off + j + e] + v;
+      }
     });
-    if (lane == 0) gcounts[k] += cnt;
+    if (!overwrite && lane == 0) gcounts[(size_t)b * K + k] += cnt;
   }
 }
 
@@ -334,15 +350,18 @@ int launch_finalize(const float *sums, const float *first, int pieces, const int
 }
 
 int launch_accumulate(const float *sums, const float *first, int pieces, const int32_t *counts,
-                      const int32_t *offsets, int K, int d, float *gsum, int32_t *gcounts,
-                      cudaStream_t s) {
+                      const int32_t *offsets, int B, int K, int d, float *gsum, int32_t *gcounts,
+                      bool overwrite, cudaStream_t s) {
   unsigned g = blocks_for(K);
   const unsigned cap = (unsigned)num_sms() * 8;
   if (g > cap) g = cap;
+  const dim3 grid(g, (unsigned)B);
   if (d % 4 == 0)
-    k_accumulate<true><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, K, d, gsum, gcounts);
+    k_accumulate<true><<<grid, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, K, d, gsum,
+                                                            gcounts, overwrite ? 1 : 0);
   else
-    k_accumulate<false><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, K, d, gsum, gcounts);
+    k_accumulate<false><<<grid, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, K, d, gsum,
+                                                             gcounts, overwrite ? 1 : 0);
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;

@@ -57,6 +57,7 @@ struct Workspace {
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
   cudaEvent_t shift_ev = nullptr;  // the max-shift copy of the Lloyd loop has landed
+  long long stream_job = 0;        // chunks streamed so far (selects the chunk buffer)
 };
 
 // Status plumbing (thread-local last-error text).
@@ -112,10 +113,11 @@ int launch_finalize(const float *sums, const float *first, int pieces, const int
                     const int32_t *offsets, float *centers, void *ch, void *cnx, int dtype, int B,
                     int K, int d, long long Kpad, unsigned *maxshift, bool from_pieces, int *err,
                     cudaStream_t s);
-// streamed path: gsum[k] += segment sum of one chunk, gcounts[k] += counts[k].
+// per-cluster totals of the segment partials of B batches: gsum[b][k] = the
+// segment sum (overwrite) or gsum[b][k] += it and gcounts[b][k] += counts[b][k].
 int launch_accumulate(const float *sums, const float *first, int pieces, const int32_t *counts,
-                      const int32_t *offsets, int K, int d, float *gsum, int32_t *gcounts,
-                      cudaStream_t s);
+                      const int32_t *offsets, int B, int K, int d, float *gsum, int32_t *gcounts,
+                      bool overwrite, cudaStream_t s);
 
 int launch_assign_f32(const float *x, const float *c, int B, long long N, int K, int d,
                       int32_t *ids, cudaStream_t s);

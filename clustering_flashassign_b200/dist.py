@@ -1,0 +1,102 @@
+"""Data-parallel Lloyd: the points of every batch split into contiguous blocks, one per rank.
+
+The pages' large-N path splits the N points into contiguous block
+partitions, one per GPU; each GPU runs its own assign and partial update over
+its block, the partial centroid sums and counts are reduced over the GPUs,
+and the new centroids are the same everywhere ("flash-kmeans and the return
+of exact K-Means on the GPU", section "Multi-GPU scaling without a NCCL
+dependency").  Here every rank is one process driving one GPU; the exchange
+is one all-reduce of the sums (B*K*d fp32) and one of the counts (B*K int32)
+per iteration through torch.distributed (NCCL over NVLink / NVSwitch), and
+every rank then runs the same finalize, so the centroids stay identical
+without a broadcast.  Each per-rank step is one call into libfk
+(fk_lloyd_step_partial, fk_update_finalize); a rank's block may sit in device
+memory or in pinned host memory (then it is streamed in chunks).
+
+    n0, n1 = block_of(N, rank, world)
+    iters = lloyd_data_parallel(x[:, n0:n1], init, max_iter, tol, ids, centers)
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+def block_of(N: int, rank: int, world: int) -> tuple[int, int]:
+    """[n0, n1): the contiguous block of rank `rank`; the first N % world ranks
+    hold one point more than the others."""
+    base, extra = divmod(N, world)
+    n0 = rank * base + min(rank, extra)
+    return n0, n0 + base + (1 if rank < extra else 0)
+
+
+class CudaSteps:
+    """The per-rank steps of lloyd_data_parallel, each one call into libfk."""
+
+    def __init__(self, stream=None, chunk_points: int = 0):
+        from . import fk_init_centers, fk_lloyd_step_partial, fk_point_norms, fk_update_finalize
+        self._init, self._partial = fk_init_centers, fk_lloyd_step_partial
+        self._norms, self._final = fk_point_norms, fk_update_finalize
+        self.stream, self.chunk_points = stream, chunk_points
+
+    def point_norms(self, x):
+        # fp16 / bf16 points resident on the device: ||x||^2 once per run
+        if x.dtype == torch.float32 or not x.is_cuda:
+            return None
+        xn = torch.empty(x.shape[:2], dtype=torch.float32, device=x.device)
+        return self._norms(x, xn, stream=self.stream)
+
+    def init_centers(self, init, centers):
+        self._init(init, centers, stream=self.stream)
+
+    def partial(self, x, xn, centers_dt, ids, sums, counts):
+        self._partial(x, xn, centers_dt, ids, sums, counts, stream=self.stream,
+                      chunk_points=self.chunk_points)
+
+    def finalize(self, sums, counts, centers, centers_dt, shift, dtype):
+        self._final(sums, counts, centers, centers_dt, shift, dtype=dtype, stream=self.stream)
+
+
+def lloyd_data_parallel(x: torch.Tensor, init_centers: torch.Tensor, max_iter: int, tol: float,
+                        ids: torch.Tensor, centers: torch.Tensor, group=None, steps=None) -> int:
+    """Lloyd's iterations over this rank's block of points.
+
+    x             (B, n, d): this rank's block (device or pinned host memory).
+    init_centers  (B, K, d) in x's dtype on this rank's device, identical on every rank.
+    ids           (B, n) int32 out (device): the block's assignment of the last iteration.
+    centers       (B, K, d) out (device): the centroids of the last update, identical on
+                  every rank.
+    group         torch.distributed group of the ranks (default: the world, when a
+                  process group is initialised; otherwise this process alone).
+    Stops after max_iter iterations or when the max centroid shift is below tol (strict);
+    every rank sees the same shift, so every rank stops after the same iteration and takes
+    the same collective steps.  Returns the number of iterations run.
+    """
+    steps = steps or CudaSteps()
+    B, _, d = x.shape
+    K = init_centers.shape[1]
+    dev = centers.device
+    reduce = dist.is_available() and dist.is_initialized()
+    sums = torch.empty((B, K, d), dtype=centers.dtype, device=dev)
+    counts = torch.empty((B, K), dtype=torch.int32, device=dev)
+    shift = torch.zeros((1,), dtype=centers.dtype, device=dev)
+    steps.init_centers(init_centers, centers)
+    low = x.dtype in (torch.float16, torch.bfloat16)
+    # the assign takes centroids in x's dtype: the initial ones first, then the
+    # rounded copy every finalize writes (fp32 points: the fp32 centroids)
+    centers_dt = torch.empty_like(init_centers) if low else None
+    cur = init_centers if low else centers
+    xn = steps.point_norms(x)
+    it = 0
+    while it < max_iter:
+        steps.partial(x, xn, cur, ids, sums, counts)
+        if reduce:
+            dist.all_reduce(sums, op=dist.ReduceOp.SUM, group=group)
+            dist.all_reduce(counts, op=dist.ReduceOp.SUM, group=group)
+        steps.finalize(sums, counts, centers, centers_dt, shift, x.dtype)
+        it += 1
+        if low:
+            cur = centers_dt
+        if tol > 0 and float(shift.item()) < tol:
+            break
+    return it

@@ -173,6 +173,78 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
              const fk_options *opts);
 
 /*
+ * Data-parallel Lloyd over point blocks (one block of points per rank).
+ * The pages' large-N path splits the N points of a batch into contiguous
+ * blocks, one per GPU; every GPU runs its own assign and partial update,
+ * the partial centroid sums and counts are summed across the GPUs, and every
+ * GPU then divides ("flash-kmeans and the return of exact K-Means on the
+ * GPU", section "Multi-GPU scaling without a NCCL dependency": contiguous
+ * block partitions, per-GPU double-buffered pipelines, reduction of the
+ * partial sums and counts).  These four calls are the per-rank pieces; the
+ * exchange between them (an all-reduce of `sums` and `counts`) belongs to
+ * the caller's communication layer.  One iteration on every rank:
+ *     fk_lloyd_step_partial(block, centers_dt) -> ids, sums, counts
+ *     sum sums and counts over the ranks
+ *     fk_update_finalize(sums, counts) -> centers, centers_dt, max_shift
+ * With identical totals every rank computes identical centroids.
+ */
+
+/*
+ * fk_point_norms -- xn[b,i] = ||x[b,i]||^2 in fp32 (fp16 / bf16 points):
+ * the point-side term the tensor-core assign ranks with.  The points of a
+ * Lloyd run do not change, so a caller computes them once and passes them
+ * to every fk_lloyd_step_partial on the same points.
+ *   x (B, N, d) in dtype, device.  xn (B, N) fp32 out, device.
+ *   fp32 points: FK_EUNSUPPORTED (that assign does not use them).
+ */
+int fk_point_norms(const void *x, int B, long long N, int d, int dtype, float *xn,
+                   fk_stream_t stream);
+
+/*
+ * fk_init_centers -- centers[b,k,:] = init[b,k,:] widened to fp32 (exact):
+ * the fp32 master copy the first fk_update_finalize starts from.
+ *   init (B, K, d) in dtype, device.  centers (B, K, d) fp32 out, device.
+ */
+int fk_init_centers(const void *init, int B, int K, int d, int dtype, float *centers,
+                    fk_stream_t stream);
+
+/*
+ * fk_lloyd_step_partial -- the local half of one data-parallel Lloyd
+ * iteration on this rank's block of points: ids = FlashAssign(x, centers_dt)
+ * (step a1, as fk_assign), then the sort-inverse reduction of the block
+ * without the division (steps a2-a5): sums[b,k,:] = sum of the block's points
+ * with id k (fp32), counts[b,k] = their number; an empty cluster gets zeros.
+ *   shape       the block: N = this rank's points per batch.
+ *   x           (B, N, d) in dtype: device memory, or pinned host memory
+ *               (then streamed in chunks of opts->chunk_points, double-
+ *               buffered, as fk_lloyd's streamed mode).
+ *   xn          nullable (B, N) fp32, device: fk_point_norms of x (used for
+ *               device-resident fp16 / bf16 points with d <= 128; else ignored).
+ *   centers_dt  (B, K, d) in dtype, device: the centroids to assign against
+ *               (for fp32 the fp32 centroids themselves).
+ *   ids         (B, N) int32 out, device.
+ *   sums        (B, K, d) fp32 out, device.  counts (B, K) int32 out, device.
+ *   opts        nullable; only chunk_points is read.
+ * Pageable host x returns FK_EINVAL.  The call is asynchronous.
+ */
+int fk_lloyd_step_partial(const fk_shape *shape, const void *x, const float *xn,
+                          const void *centers_dt, int32_t *ids, float *sums, int32_t *counts,
+                          fk_stream_t stream, const fk_options *opts);
+
+/*
+ * fk_update_finalize -- the division of the update from summed partials:
+ * centers[b,k] = sums[b,k] / counts[b,k] where counts[b,k] > 0, else
+ * unchanged; centers_dt receives the centroids rounded to dtype (nearest
+ * even) for the next assign; max_shift = max over b,k of ||new - old||_2.
+ *   sums (B, K, d) fp32, counts (B, K) int32, device (totals over the ranks).
+ *   centers     (B, K, d) fp32, device, in: previous centroids, out: new.
+ *   centers_dt  (B, K, d) in dtype, device, out (ignored, may be NULL, for fp32).
+ *   max_shift   nullable device float.
+ */
+int fk_update_finalize(const float *sums, const int32_t *counts, int B, int K, int d, int dtype,
+                       float *centers, void *centers_dt, float *max_shift, fk_stream_t stream);
+
+/*
  * fk_assign_noalloc -- fk_assign for callers that cannot allocate device
  * memory (no counterpart in the paper; it is an interface addition).
  * Same arguments, layouts and result as fk_assign.  Callers that run under an
