@@ -60,10 +60,17 @@ def load_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the FlashAssign kernel's own sources (the kernel file, the sm_100
+    PTX layer, the norm-row arithmetic) and of the constants it takes from the
+    internal header, so host-side declarations there do not count as a change."""
     h = hashlib.sha256()
-    for name in ["fk_assign_tc.cu", "fk_sm100.cuh", "fk_internal.h"]:
-        with open(os.path.join(ROOT, "clustering_flashassign_b200", "csrc", name), "rb") as f:
+    csrc = os.path.join(ROOT, "clustering_flashassign_b200", "csrc")
+    for name in ["fk_assign_tc.cu", "fk_sm100.cuh", "fk_norms.cuh"]:
+        with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
+    with open(os.path.join(csrc, "fk_internal.h")) as f:
+        consts = [ln for ln in f if re.match(r"\s*(constexpr|enum|inline)\b", ln)]
+    h.update("".join(consts).encode())
     return h.hexdigest()[:16]
 
 
