@@ -100,11 +100,35 @@ int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long
                          d, Kpad, ws->maxshift, true, ws->err, s);
 }
 
+// fp32 on the tensor cores: the centroids' [hi | lo | hi] rows and tf32 norm
+// rows every call; the points' [hi | hi | lo] rows from x3 when the caller
+// prepared them (a Lloyd run does it once), else built here.
+int assign_f32_tc(Workspace *ws, const float *x, const float *c, const float *x3, int B, long long N,
+                  int K, int d, long long Kpad, int32_t *ids, cudaStream_t s, uint32_t *hist) {
+  const int d3 = 3 * d;
+  if (!x3) {
+    FK_TRY(ensure(ws->x3, (size_t)B * N * d3 * sizeof(float)));
+    FK_TRY(launch_split3(x, (long long)B * N, d, (float *)ws->x3.p, false, s));
+    x3 = (const float *)ws->x3.p;
+  }
+  FK_TRY(ensure(ws->c3, (size_t)B * K * d3 * sizeof(float)));
+  FK_TRY(launch_split3(c, (long long)B * K, d, (float *)ws->c3.p, true, s));
+  FK_TRY(ensure(ws->cn, ext_bytes(B, Kpad)));
+  FK_TRY(launch_prep_ext_f32(c, B, K, d, Kpad, ws->cn.p, s));
+  return launch_assign_tc(x3, ws->c3.p, ws->cn.p, nullptr, FK_F32, B, N, K, d3, Kpad, ids, ws->err, s,
+                          hist);
+}
+
 int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const void *cnx,
                        const float *xn, int B, long long N, int K, int d, int dtype, long long Kpad,
-                       int32_t *ids, cudaStream_t s, uint32_t *hist = nullptr) {
+                       int32_t *ids, cudaStream_t s, uint32_t *hist = nullptr,
+                       const float *x3 = nullptr) {
   PhaseTimer t(PH_ASSIGN, s);
-  if (dtype == FK_F32) return launch_assign_f32((const float *)x, (const float *)cdt, B, N, K, d, ids, s);
+  if (dtype == FK_F32) {
+    if (use_tf32(K, d))
+      return assign_f32_tc(ws, (const float *)x, (const float *)cdt, x3, B, N, K, d, Kpad, ids, s, hist);
+    return launch_assign_f32((const float *)x, (const float *)cdt, B, N, K, d, ids, s);
+  }
   return launch_assign_tc(x, cdt, cnx, xn, dtype, B, N, K, d, Kpad, ids, ws->err, s, hist);
 }
 
@@ -373,7 +397,7 @@ int fk_lloyd_step_partial(const fk_shape *shape, const void *x, const float *xn,
     return streamed_pass(ws, sh, (const char *)x, chunk, centers_dt, cnx, ids, sums, counts, s);
   }
   // With K <= 4096 the assign counts every id into the sort's tile histogram.
-  const bool fuse = tc && sort_single_pass(K);
+  const bool fuse = (tc || use_tf32(K, d)) && sort_single_pass(K);
   uint32_t *hist = nullptr;
   if (fuse) {
     const size_t hist_bytes = sort_table_bytes(B, N, K);
@@ -498,9 +522,17 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
       idbuf[1] = (int32_t *)ws->ids_alt.p;
       if (!ws->shift_ev) FK_CUDA(cudaEventCreateWithFlags(&ws->shift_ev, cudaEventDisableTiming));
     }
+    // fp32 on the tensor cores: the points' [hi | hi | lo] rows once per call
+    const bool tc32 = dtype == FK_F32 && use_tf32(K, d);
+    const float *x3 = nullptr;
+    if (tc32) {
+      FK_TRY(ensure(ws->x3, (size_t)B * N * 3 * d * sizeof(float)));
+      FK_TRY(launch_split3((const float *)xdev, (long long)B * N, d, (float *)ws->x3.p, false, s));
+      x3 = (const float *)ws->x3.p;
+    }
     // With K <= 4096 the tensor-core assign also counts every id into the
     // sort's tile histogram, so the sort starts at its scan.
-    const bool fuse = dtype != FK_F32 && sort_single_pass(K);
+    const bool fuse = (dtype != FK_F32 || tc32) && sort_single_pass(K);
     uint32_t *hist = nullptr;
     const size_t hist_bytes = sort_table_bytes(B, N, K);
     if (fuse) {
@@ -509,7 +541,7 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
     }
     auto assign = [&](int32_t *out) -> int {
       if (hist) FK_CUDA(cudaMemsetAsync(hist, 0, hist_bytes, s));
-      return do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, out, s, hist);
+      return do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, out, s, hist, x3);
     };
     int cur = 0;
     if (max_iter > 0) FK_TRY(assign(idbuf[0]));

@@ -140,14 +140,26 @@ __device__ __forceinline__ float key_hi(float key) {
   return __uint_as_float(__float_as_uint(key) & kKeyMask);
 }
 
-// Stores one 16-element norm row at row r of a K-major 32-byte-swizzled tile:
-// 16-byte chunk q of row r sits at r * 32 + ((q ^ ((r >> 2) & 1)) * 16).
+// One MMA step of the element type's kind: kind::f16 for fp16 / bf16 (K = 16),
+// kind::tf32 for fp32 (K = 8); either way 32 bytes of every operand row.
 template <typename T>
-__device__ __forceinline__ void store_ext_row_sw32(uint8_t *tile, int r, const T (&row)[kExt]) {
+__device__ __forceinline__ void mma_t(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                      uint32_t accumulate) {
+  if constexpr (sizeof(T) == 4) mma_tf32(d_tmem, a_desc, b_desc, idesc, accumulate);
+  else mma_f16(d_tmem, a_desc, b_desc, idesc, accumulate);
+}
+
+// Stores one 32-byte norm row at row r of a K-major 32-byte-swizzled tile:
+// 16-byte chunk q of row r sits at r * 32 + ((q ^ ((r >> 2) & 1)) * 16).
+__device__ __forceinline__ void store_row32_sw32(uint8_t *tile, int r, const void *row) {
   const int flip = (r >> 2) & 1;
   uint4 *p = reinterpret_cast<uint4 *>(tile + r * 32);
-  p[flip] = *reinterpret_cast<const uint4 *>(&row[0]);
-  p[flip ^ 1] = *reinterpret_cast<const uint4 *>(&row[8]);
+  p[flip] = reinterpret_cast<const uint4 *>(row)[0];
+  p[flip ^ 1] = reinterpret_cast<const uint4 *>(row)[1];
+}
+template <typename T>
+__device__ __forceinline__ void store_ext_row_sw32(uint8_t *tile, int r, const T (&row)[kExt]) {
+  store_row32_sw32(tile, r, row);
 }
 
 // a0 += lo(v)^2, a1 += hi(v)^2 for two packed 16-bit values, fp32 accumulation
@@ -207,6 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_flash_assign(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmc,
                    const __grid_constant__ CUtensorMap tme, const TcArgs a) {
   using L = Layout<RESIDENT, KB, STAGES>;
+  constexpr int kBlockE = 128 / (int)sizeof(T);  // elements per 128-byte K-block row
+  static_assert(!RESIDENT || sizeof(T) == 2, "the resident-tile variant is for 16-bit points");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -268,9 +282,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (!RESIDENT && warp == kNormWarp) {
     // split-d: one constant point-side row (the -S_e that multiply ||c||^2's digits)
-    T row[kExt];
-    ext_point_row<T, false>(0.f, row);
-    for (int r = lane; r < kTileM; r += 32) store_ext_row_sw32<T>(smem + L::kAExtOff, r, row);
+    if constexpr (sizeof(T) == 4) {
+      alignas(16) float row[kExtF32];
+      ext_point_row_f32(row);
+      for (int r = lane; r < kTileM; r += 32) store_row32_sw32(smem + L::kAExtOff, r, row);
+    } else {
+      alignas(16) T row[kExt];
+      ext_point_row<T, false>(0.f, row);
+      for (int r = lane; r < kTileM; r += 32) store_ext_row_sw32<T>(smem + L::kAExtOff, r, row);
+    }
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -295,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = tile / a.tiles_per_batch;
         const int row0 = (tile % a.tiles_per_batch) * kTileM;
         for (int kb = 0; kb < KB; ++kb)
-          tma_load_3d(&tmx, x_base + (xb * KB + kb) * kXBlockBytes, xfull(xb), kb * kBlockK, row0, b);
+          tma_load_3d(&tmx, x_base + (xb * KB + kb) * kXBlockBytes, xfull(xb), kb * kBlockE, row0, b);
         ++g;
         return true;
       };
@@ -310,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dst = st_base + s * L::kStageBytes;
             mbar_arrive_expect_tx(full(s), L::kStageBytes);
             for (int kb = 0; kb < KB; ++kb)
-              tma_load_3d(&tmc, dst + kb * kCBlockBytes, full(s), kb * kBlockK, c * kChunkN, b);
+              tma_load_3d(&tmc, dst + kb * kCBlockBytes, full(s), kb * kBlockE, c * kChunkN, b);
             tma_load_3d(&tme, dst + KB * kCBlockBytes, full(s), 0, c * kChunkN, b);
             ++f;
           } else {  // this chunk's centroid norm rows (used by the chunk's last MMA step)
@@ -325,8 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
             const uint32_t dst = st_base + s * L::kStageBytes;
             mbar_arrive_expect_tx(full(s), kXBlockBytes + kCBlockBytes);
-            tma_load_3d(&tmx, dst, full(s), kb * kBlockK, row0, b);
-            tma_load_3d(&tmc, dst + kXBlockBytes, full(s), kb * kBlockK, c * kChunkN, b);
+            tma_load_3d(&tmx, dst, full(s), kb * kBlockE, row0, b);
+            tma_load_3d(&tmc, dst + kXBlockBytes, full(s), kb * kBlockE, c * kChunkN, b);
             ++f;
           }
           if (RESIDENT && ok && c == 0 && tile + (int)gridDim.x < a.total_tiles)
@@ -377,11 +397,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t b_addr = stage + kb * kCBlockBytes;
 #pragma unroll
               for (int k = 0; k < kBlockK / 16; ++k)
-                mma_f16(d_tmem, desc_k_sw128(a_addr + k * 32), desc_k_sw128(b_addr + k * 32), a.idesc,
+                mma_t<T>(d_tmem, desc_k_sw128(a_addr + k * 32), desc_k_sw128(b_addr + k * 32), a.idesc,
                         (kb | k) != 0 ? 1u : 0u);
             }
             // the norm step: acc += A_ext . B_ext (fk_norms.cuh)
-            mma_f16(d_tmem, desc_k_sw32(a_ext), desc_k_sw32(stage + KB * kCBlockBytes), a.idesc, 1u);
+            mma_t<T>(d_tmem, desc_k_sw32(a_ext), desc_k_sw32(stage + KB * kCBlockBytes), a.idesc, 1u);
             mma_commit(empty(s));  // frees the stage once these MMAs have read it
             ++f;
             mma_commit(accfull(ab));  // accumulator ready for the epilogue
@@ -397,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t b_addr = RESIDENT ? stage : stage + kXBlockBytes;
 #pragma unroll
             for (int k = 0; k < kBlockK / 16; ++k)
-              mma_f16(d_tmem, desc_k_sw128(a_addr + k * 32), desc_k_sw128(b_addr + k * 32), a.idesc,
+              mma_t<T>(d_tmem, desc_k_sw128(a_addr + k * 32), desc_k_sw128(b_addr + k * 32), a.idesc,
                       (kb | k) != 0 ? 1u : 0u);
             mma_commit(empty(s));  // frees the stage once these MMAs have read it
             ++f;
@@ -411,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int es = e % kExtSlots;
           if (!mbar_wait(efull(es), (e / kExtSlots) & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
-          mma_f16(d_tmem, desc_k_sw32(a_ext), desc_k_sw32(bext_base + es * kBExtBytes), a.idesc, 1u);
+          mma_t<T>(d_tmem, desc_k_sw32(a_ext), desc_k_sw32(bext_base + es * kBExtBytes), a.idesc, 1u);
           mma_commit(eempty(es));
           ++e;
           mma_commit(accfull(ab));  // accumulator ready for the epilogue
@@ -428,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kNormWarp) {
     // ------------------------------------------------------------ point norms
-    if (RESIDENT) {
+    if constexpr (RESIDENT) {
       uint32_t g = 0;
       for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++g) {
         const int xb = g & 1;
@@ -654,18 +674,23 @@ int get_encoder(EncodeTiledFn *out) {
   return FK_OK;
 }
 
-// (inner, rows, B) tensor of 16-bit elements, box (box_inner, box_rows, 1).
+// (inner, rows, B) tensor of dtype's elements (fp32 for FK_F32, else 16-bit),
+// box (box_inner, box_rows, 1).
 int encode_3d(CUtensorMap *map, const void *base, int dtype, int inner, long long rows, int B,
               int box_inner, int box_rows, CUtensorMapSwizzle swz) {
   EncodeTiledFn enc;
   FK_TRY(get_encoder(&enc));
+  const cuuint64_t es = dtype == FK_F32 ? 4 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)B};
-  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)rows * inner * 2};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * es, (cuuint64_t)rows * inner * es};
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, dtype == FK_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                   3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapDataType ty = dtype == FK_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : dtype == FK_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = enc(map, ty, 3, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(FK_ECUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
   return FK_OK;
 }
@@ -690,8 +715,10 @@ template <typename T>
 int launch_typed(const CUtensorMap &tmx, const CUtensorMap &tmc, const CUtensorMap &tme,
                  const TcArgs &a, int grid, cudaStream_t s) {
   // resident stages hold whole chunks: 4 x 40 KB (d <= 64) or 2 x 72 KB (d <= 128)
-  if (a.kblocks == 1) return launch_variant<T, true, 1, 4>(tmx, tmc, tme, a, grid, s);
-  if (a.kblocks == 2) return launch_variant<T, true, 2, 2>(tmx, tmc, tme, a, grid, s);
+  if constexpr (sizeof(T) == 2) {
+    if (a.kblocks == 1) return launch_variant<T, true, 1, 4>(tmx, tmc, tme, a, grid, s);
+    if (a.kblocks == 2) return launch_variant<T, true, 2, 2>(tmx, tmc, tme, a, grid, s);
+  }
   return launch_variant<T, false, 1, 4>(tmx, tmc, tme, a, grid, s);
 }
 
@@ -705,10 +732,14 @@ int launch_point_norms(const void *x, int dtype, long long rows, int d, float *x
 int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float *xn, int dtype,
                      int B, long long N, int K, int d, long long Kpad, int32_t *ids, int *err,
                      cudaStream_t s, uint32_t *hist) {
+  // K-blocks are 128-byte rows: 64 16-bit elements or 32 fp32 (read as tf32);
+  // norm rows are 32 bytes: 16 or 8 elements
+  const int blk = dtype == FK_F32 ? 32 : kBlockK;
+  const int ext = dtype == FK_F32 ? kExtF32 : kExt;
   CUtensorMap tmx, tmc, tme;
-  FK_TRY(encode_3d(&tmx, x, dtype, d, N, B, kBlockK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B));
-  FK_TRY(encode_3d(&tmc, ch, dtype, d, K, B, kBlockK, kChunkN, CU_TENSOR_MAP_SWIZZLE_128B));
-  FK_TRY(encode_3d(&tme, cnx, dtype, kExt, Kpad, B, kExt, kChunkN, CU_TENSOR_MAP_SWIZZLE_32B));
+  FK_TRY(encode_3d(&tmx, x, dtype, d, N, B, blk, kTileM, CU_TENSOR_MAP_SWIZZLE_128B));
+  FK_TRY(encode_3d(&tmc, ch, dtype, d, K, B, blk, kChunkN, CU_TENSOR_MAP_SWIZZLE_128B));
+  FK_TRY(encode_3d(&tme, cnx, dtype, ext, Kpad, B, ext, kChunkN, CU_TENSOR_MAP_SWIZZLE_32B));
   TcArgs a;
   a.N = (int)N;
   a.K = K;
@@ -719,13 +750,14 @@ int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float
   if (total > 0x7fffffffLL) return set_error(FK_EUNSUPPORTED, "too many point tiles");
   a.total_tiles = (int)total;
   a.nchunks = (K + kChunkN - 1) / kChunkN;
-  a.kblocks = (d + kBlockK - 1) / kBlockK;
+  a.kblocks = (d + blk - 1) / blk;
   a.xn = xn;
   a.ids = ids;
   a.err = err;
-  a.idesc = sm100::idesc_f16(dtype == FK_BF16 ? 1u : 0u, kTileM, kChunkN);
+  a.idesc = sm100::idesc_f32acc(dtype == FK_F32 ? 2u : dtype == FK_BF16 ? 1u : 0u, kTileM, kChunkN);
   int grid = num_sms();
   if (total < grid) grid = (int)total;
+  if (dtype == FK_F32) return launch_typed<float>(tmx, tmc, tme, a, grid, s);
   if (dtype == FK_BF16) return launch_typed<__nv_bfloat16>(tmx, tmc, tme, a, grid, s);
   return launch_typed<__half>(tmx, tmc, tme, a, grid, s);
 }

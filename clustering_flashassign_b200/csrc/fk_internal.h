@@ -54,6 +54,7 @@ struct Workspace {
   float *h_maxshift = nullptr;    // pinned host mirror
   DevBuf cn, ch, sums, first, counts, offsets, table, digit_off, kv, keys_b, vals_b;
   DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2], gsum, gcounts, xn, ids_alt;
+  DevBuf x3, c3;                  // 3xTF32 operands of the fp32 tensor-core assign
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
   cudaEvent_t shift_ev = nullptr;  // the max-shift copy of the Lloyd loop has landed
@@ -121,6 +122,14 @@ int launch_accumulate(const float *sums, const float *first, int pieces, const i
 
 int launch_assign_f32(const float *x, const float *c, int B, long long N, int K, int d,
                       int32_t *ids, cudaStream_t s);
+// fp32 on the tensor cores (3xTF32, fk_tf32.cu): used when d % 4 == 0 and
+// K * d >= kTf32MinKd; smaller problems stay on the CUDA-core kernel.
+constexpr long long kTf32MinKd = 16384;
+bool use_tf32(int K, int d);
+// dst (rows, 3d) = [hi | hi | lo] (points) or [hi | lo | hi] (centroids) of src (rows, d).
+int launch_split3(const float *src, long long rows, int d, float *dst, bool centroids, cudaStream_t s);
+// tf32 norm rows (B, Kpad, 8) fp32 of the fp32 centroids c (B, K, d).
+int launch_prep_ext_f32(const float *c, int B, int K, int d, long long Kpad, void *cnx, cudaStream_t s);
 // cnx: extension rows (B, Kpad, 16) in dtype from launch_prep_cn / finalize;
 // xn: ||x||^2 per point (B, N) from launch_point_norms, or NULL (the kernel
 // then computes it from its shared copy of each point tile).

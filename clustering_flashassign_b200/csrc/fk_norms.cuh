@@ -144,4 +144,38 @@ __device__ __forceinline__ bool ext_point_row(float xn2, T (&row)[kExt]) {
   return clamped;
 }
 
+// tf32 (fp32 points on the tensor cores, kind::tf32, exact mode only): a row
+// is 8 fp32 values (32 bytes, one K = 8 step).  ||c||^2 / 2 is split into
+// three tf32 digits (the value truncated to 10 fraction bits, then the exact
+// remainder truncated the same way, then the rest, which has at most 2
+// significant bits left), so the digits sum back to the fp32 value exactly.
+//   B side: [t0, t1, t2, 0, 0, 0, 0, 0]   A side: [-1, -1, -1, 0, 0, 0, 0, 0]
+// giving acc = x.c - ||c||^2 / 2.  A padded centroid gets t0 = 2^100.
+constexpr int kExtF32 = 8;
+
+__device__ __forceinline__ float tf32_trunc(float v) {
+  return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+}
+
+__device__ __forceinline__ void ext_centroid_row_f32(float cn, bool real, float (&row)[kExtF32]) {
+#pragma unroll
+  for (int e = 0; e < kExtF32; ++e) row[e] = 0.f;
+  if (!real) {
+    row[0] = 1267650600228229401496703205376.f;  // 2^100
+    return;
+  }
+  float r = 0.5f * cn;
+#pragma unroll
+  for (int e = 0; e < 3; ++e) {
+    const float t = e < 2 ? tf32_trunc(r) : r;
+    row[e] = t;
+    r -= t;  // exact: t holds leading bits of r
+  }
+}
+
+__device__ __forceinline__ void ext_point_row_f32(float (&row)[kExtF32]) {
+#pragma unroll
+  for (int e = 0; e < kExtF32; ++e) row[e] = e < 3 ? -1.f : 0.f;
+}
+
 }  // namespace fk

@@ -107,7 +107,7 @@ int release_device_workspaces() {
     }
     Workspace *ws = it->second;
     DevBuf *bufs[] = {&ws->cn, &ws->ch, &ws->sums, &ws->first, &ws->counts, &ws->offsets,
-                      &ws->table, &ws->digit_off, &ws->kv, &ws->keys_b,
+                      &ws->table, &ws->digit_off, &ws->kv, &ws->x3, &ws->c3, &ws->keys_b,
                       &ws->vals_b, &ws->xres, &ws->init_dev, &ws->ids_dev, &ws->centers_dev,
                       &ws->chunk[0], &ws->chunk[1], &ws->gsum, &ws->gcounts, &ws->xn, &ws->ids_alt};
     for (DevBuf *b : bufs) free_buf(*b);

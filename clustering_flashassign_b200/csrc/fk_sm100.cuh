@@ -138,6 +138,18 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::tf32 (32-bit containers read as
+// tf32, fp32 accumulate); K = 8 per instruction, 32 bytes of each row.
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on `bar` when every tcgen05 op issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -191,9 +203,10 @@ __device__ __forceinline__ uint64_t desc_k_sw32(uint32_t saddr) {
   return desc;
 }
 
-// Instruction descriptor of kind::f16 with fp32 accumulation, A and B K-major.
-// ab_fmt: 0 = fp16, 1 = bf16 (A and B always share it).
-__host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_fmt, uint32_t M, uint32_t N) {
+// Instruction descriptor with fp32 accumulation, A and B K-major.  ab_fmt
+// (A and B always share it): 0 = fp16, 1 = bf16 (kind::f16), 2 = tf32
+// (kind::tf32).
+__host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t ab_fmt, uint32_t M, uint32_t N) {
   return (1u << 4)              // D format fp32
          | (ab_fmt << 7)        // A format
          | (ab_fmt << 10)       // B format

@@ -81,7 +81,13 @@ def test_flash_assign_exact_ties_take_lowest_index():
     assert ids2[:, :3].cpu().numpy().tolist() == [[3, 100, 0]] * B
 
 
-@pytest.mark.parametrize("B,N,K,d", [(1, 8192, 64, 32), (2, 1000, 37, 5), (1, 300, 70, 100)])
+@pytest.mark.parametrize("B,N,K,d", [
+    (1, 8192, 64, 32), (2, 1000, 37, 5), (1, 300, 70, 100),   # CUDA cores (K * d < 16384 or d % 4)
+    (2, 3000, 300, 64),      # tensor cores, 3xTF32: 192-wide extended rows, six K-blocks
+    (1, 1000, 600, 100),     # ragged last K-block (300 = 9 x 32 + 12), ragged chunk
+    (3, 300, 257, 128),      # ragged point tile, one centroid past a chunk
+    (1, 2048, 1024, 2048),   # the large-D fp32 shape of the pages' FlashKMeans example
+])
 def test_fp32_assign_matches_oracle(B, N, K, d):
     import clustering_flashassign_b200 as fk
     x, idx, c0 = case(B, N, K, d, "f32", mean_std=4.0)

@@ -16,7 +16,8 @@ def round_dtype(c32: np.ndarray, dtype: str) -> np.ndarray:
 
 
 @pytest.mark.parametrize("B,N,K,d,dtype", [(2, 3000, 200, 128, "f16"), (2, 2500, 150, 64, "bf16"),
-                                           (1, 4000, 64, 32, "f32"), (1, 1500, 300, 256, "bf16")])
+                                           (1, 4000, 64, 32, "f32"), (1, 1500, 300, 256, "bf16"),
+                                           (1, 3000, 256, 128, "f32")])   # fp32 on the tensor cores
 def test_lockstep_iterations(B, N, K, d, dtype):
     """Each iteration: oracle assign with the GPU's dtype centroids, oracle
     update with the GPU's ids; the GPU continues from its own centroids."""
@@ -40,11 +41,13 @@ def test_lockstep_iterations(B, N, K, d, dtype):
     assert flips <= B * N * 1e-3
 
 
-@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
-def test_lloyd_equals_its_steps(dtype):
-    """fk_lloyd == fk_assign / fk_update with centroids rounded to dtype in between."""
+@pytest.mark.parametrize("dtype,K", [("f16", 100), ("bf16", 100), ("f32", 100), ("f32", 300)])
+def test_lloyd_equals_its_steps(dtype, K):
+    """fk_lloyd == fk_assign / fk_update with centroids rounded to dtype in between
+    (fp32 with K = 300 runs on the tensor cores: fk_lloyd splits the points once,
+    fk_assign on every call)."""
     import clustering_flashassign_b200 as fk
-    B, N, K, d = 2, 2000, 100, 64
+    B, N, d = 2, 2000, 64
     x, idx, c0 = case(B, N, K, d, dtype, n_comp=60, mean_std=3.0)
     xd, cd = to_dev(x, dtype), to_dev(c0, dtype)
     ids_l = torch.empty((B, N), dtype=torch.int32, device="cuda")
