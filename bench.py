@@ -220,11 +220,28 @@ def reduce_over_ranks(dist, device, to_max, to_sum):
     return [float(v) for v in tmax.tolist()], [float(v) for v in tsum.tolist()]
 
 
-def cpu_oracle_sample(x, init, w, batches, threads=0):
-    """One Lloyd iteration of the fp64 checker on `batches` of the workload."""
+# distance terms (points x centroids x d) the CPU sample may cover: about
+# 2-3 s of the fp64 checker on 16 cores
+CPU_SAMPLE_TERMS = 4e10
+
+
+def cpu_sample_points(w, batches):
+    """Points per batch of the CPU sample: all of them, or a prefix when the
+    sample would exceed CPU_SAMPLE_TERMS."""
+    terms = batches * w.N * w.K * w.d
+    if terms <= CPU_SAMPLE_TERMS:
+        return w.N
+    return max(min(w.N, 1024), int(w.N * CPU_SAMPLE_TERMS / terms))
+
+
+def cpu_oracle_sample(x, init, w, batches, threads=0, points=None):
+    """One Lloyd iteration of the fp64 checker on `batches` of the workload
+    (the first `points` points of each, all by default)."""
+    import numpy as np
+
     import oracle
     import synthdata
-    xs = x[:batches].copy()
+    xs = np.ascontiguousarray(x[:batches, :points] if points else x[:batches])
     c = synthdata.to_f64(init[:batches], w.dtype)
     t0 = time.perf_counter()
     chat = oracle.round_to(c, w.dtype)
@@ -351,7 +368,14 @@ def run_fk(args, rank, world, local_rank, dist):
     flop = 2.0 * w.B * w.N * w.K * w.d
     a_ms = prof["assign_ms"] / max(1, prof["assign_launches"])
     achieved = flop / (a_ms * 1e-3) / 1e12
-    if w.dtype == "f32":
+    tf32 = w.dtype == "f32" and w.d % 4 == 0 and w.K * w.d >= 16384
+    if tf32:
+        # fp32 on the tensor cores, 3xTF32: three tf32 passes per algorithmic flop;
+        # the tf32 peak is the measured bf16 peak times the nominal ratio 1.1 / 2.25
+        peak_t = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]) * 1.1 / 2.25
+        bound, kname = "tensor", "FlashAssign kind::tf32, 3 passes (k_flash_assign<float>)"
+        psrc = f"{src} bf16 dense sustained x 1.1/2.25 (nominal tf32 : bf16); the 3xTF32 split runs 3 tensor passes per algorithmic flop, so 1/3 is the attainable fraction"
+    elif w.dtype == "f32":
         # fp32 inputs take the SIMT kernel: peak from unit counts and the max clock
         mhz = float(peaks.get("sm_max_mhz", 1965.0))
         peak_t = 148 * 128 * 2 * mhz * 1e6 / 1e12
@@ -371,8 +395,9 @@ def run_fk(args, rank, world, local_rank, dist):
 
     import oracle
     batches = min(4, w.B)
-    cpu_t = cpu_oracle_sample(x, init, w, batches)
-    cpu_value = 1.0 / (cpu_t * w.B / batches)
+    pts = cpu_sample_points(w, batches)
+    cpu_t = cpu_oracle_sample(x, init, w, batches, points=pts)
+    cpu_value = 1.0 / (cpu_t * (w.B / batches) * (w.N / pts))
 
     line = {
         "metric": metric_for(w),
@@ -405,7 +430,10 @@ def run_fk(args, rank, world, local_rank, dist):
                     "split_from": "one extra step with an event pair around every phase",
                     "hbm_peak_gbs": hbm},
         "cpu_baseline": {"value": cpu_value, "unit": "iter/s", "cores": oracle.max_threads(), "kind": "oracle",
-                         "sample": f"one Lloyd iteration of {batches} of {w.B} batches, extrapolated"},
+                         "sample": (f"one Lloyd iteration of {batches} of {w.B} batches, extrapolated"
+                                    if pts == w.N else
+                                    f"one Lloyd iteration on the first {pts} of {w.N} points of {batches} "
+                                    f"of {w.B} batches, extrapolated x{w.B * w.N / (batches * pts):.1f}")},
         "e2e": {"value": e_iters / (e_ms * 1e-3), "unit": "iter/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
@@ -623,7 +651,7 @@ def main():
     ap.add_argument("--points", type=int, default=0, help="with --kernel-case / --workload: points per batch")
     ap.add_argument("--baselines", action="store_true",
                     help="time the materialised-distance assign and the scatter-atomic update next to libfk")
-    ap.add_argument("--workload", default="api", choices=["api", "tiny", "zipf", "splitd", "largen"],
+    ap.add_argument("--workload", default="api", choices=["api", "tiny", "zipf", "splitd", "largen", "f32large"],
                     help="api is the benchmark; the others print their own line (largen: the 64 GiB "
                          "streamed workload)")
     args = ap.parse_args()

@@ -152,6 +152,8 @@ WORKLOADS = {
     "zipf": Workload("zipf", 32, 65536, 1024, 128, "f16", 1024, 3.0, 1.2, 20, 0.0, 103, 3000),
     "splitd": Workload("splitd", 8, 32768, 4096, 1024, "bf16", 4096, 2.0, 0.0, 10, 0.0, 104, 4000),
     "largen": Workload("largen", 1, 1 << 28, 32768, 128, "f16", 32768, 4.0, 0.0, 3, 0.0, 105, 5000),
+    # the large-D fp32 shape of the pages' FlashKMeans example (d = 2048, k = 1024)
+    "f32large": Workload("f32large", 1, 1 << 19, 1024, 2048, "f32", 1024, 4.0, 0.0, 5, 0.0, 106, 6000),
 }
 
 
