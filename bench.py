@@ -617,10 +617,8 @@ def run_kernel_case(args):
 
     import clustering_flashassign_b200 as fk
     import synthdata
-    w, x, init = make_inputs(0)
-    if args.points:
-        w = synthdata.scaled(w, N=args.points)
-        x = x[:, : args.points].copy()
+    w = rank_workload(0, args.workload, **({"N": args.points} if args.points else {}))
+    x, _, init = synthdata.make(w)
     xd = torch.from_numpy(x).cuda()
     cd = torch.from_numpy(init).cuda()
     ids = torch.empty((w.B, w.N), dtype=torch.int32, device="cuda")
