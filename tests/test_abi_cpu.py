@@ -87,3 +87,28 @@ def test_binding_rejects_noncontiguous_tensors():
     x = torch.zeros(2, 16, 8, dtype=torch.float16).transpose(0, 1)
     with pytest.raises(ValueError):
         fk.fk_assign(x, torch.zeros(16, 2, 8, dtype=torch.float16), torch.zeros(16, 2, dtype=torch.int32))
+
+
+def test_data_parallel_pieces_validate_on_the_host():
+    """fk_point_norms, fk_init_centers, fk_lloyd_step_partial and fk_update_finalize
+    reject bad shapes and pointers before any device work."""
+    import clustering_flashassign_b200 as fk
+    L = fk.lib
+    p = ctypes.c_void_p(0x1000)
+    assert L.fk_point_norms(p, 1, 10, 8, fk.FK_F32, p, None) == fk.FK_EUNSUPPORTED
+    assert L.fk_point_norms(None, 1, 10, 8, fk.FK_F16, p, None) == fk.FK_EINVAL
+    assert "x is NULL" in fk.fk_last_error()
+    assert L.fk_point_norms(p, 1, 10, 12, fk.FK_F16, p, None) == fk.FK_EINVAL
+    assert L.fk_init_centers(p, 1, 0, 8, fk.FK_F16, p, None) == fk.FK_EINVAL
+    assert L.fk_init_centers(p, 1, 4, 8, fk.FK_F16, None, None) == fk.FK_EINVAL
+    shape = fk.FkShape(1, 10, 2, 8, fk.FK_F16)
+    assert L.fk_lloyd_step_partial(None, p, None, p, p, p, p, None, None) == fk.FK_EINVAL
+    assert "shape is NULL" in fk.fk_last_error()
+    assert L.fk_lloyd_step_partial(ctypes.byref(shape), p, None, p, p, None, p, None, None) == fk.FK_EINVAL
+    assert "sums is NULL" in fk.fk_last_error()
+    bad = fk.FkShape(1, 10, 11, 8, fk.FK_F16)
+    assert L.fk_lloyd_step_partial(ctypes.byref(bad), p, None, p, p, p, p, None, None) == fk.FK_EINVAL
+    assert L.fk_update_finalize(p, None, 1, 4, 8, fk.FK_F16, p, p, None, None) == fk.FK_EINVAL
+    assert "counts is NULL" in fk.fk_last_error()
+    assert L.fk_update_finalize(p, p, 1, 4, 8, 9, p, p, None, None) == fk.FK_EINVAL
+    assert "unknown dtype" in fk.fk_last_error()
