@@ -82,7 +82,8 @@ int do_update(Workspace *ws, const void *x, const int32_t *ids, int B, long long
     counts = (int32_t *)ws->counts.p;
   }
   FK_TRY(prepare_update(ws, B, N, K, d));
-  FK_CUDA(cudaMemsetAsync(ws->maxshift, 0, sizeof(unsigned), s));
+  // the max-shift word is zeroed by the sort's scan kernel (no memset between
+  // the dependent launches of the update)
   int2 *kv = (int2 *)ws->kv.p;
   int32_t *offsets = (int32_t *)ws->offsets.p;
   float *sums = (float *)ws->sums.p, *first = (float *)ws->first.p;
@@ -539,8 +540,10 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
       FK_TRY(ensure(ws->table, hist_bytes));
       hist = (uint32_t *)ws->table.p;
     }
+    // the table starts at zero; afterwards every sort's scatter zeroes the
+    // rows it has read, so no memset separates the iterations' launches
+    if (hist) FK_CUDA(cudaMemsetAsync(hist, 0, hist_bytes, s));
     auto assign = [&](int32_t *out) -> int {
-      if (hist) FK_CUDA(cudaMemsetAsync(hist, 0, hist_bytes, s));
       return do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, out, s, hist, x3);
     };
     int cur = 0;

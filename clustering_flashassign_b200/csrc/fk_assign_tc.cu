@@ -298,6 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int kblocks = RESIDENT ? KB : a.kblocks;
+  // the set-up above overlaps the previous kernel of the stream; everything
+  // below may read what it wrote
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -705,7 +708,8 @@ int launch_variant(const CUtensorMap &tmx, const CUtensorMap &tmc, const CUtenso
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc));
     attr = true;
   }
-  k_flash_assign<T, RESIDENT, KB, STAGES><<<grid, kThreads, L::kAlloc, s>>>(tmx, tmc, tme, a);
+  FK_CUDA(launch_pdl(k_flash_assign<T, RESIDENT, KB, STAGES>, dim3(grid), dim3(kThreads), L::kAlloc, s, tmx, tmc,
+                     tme, a));
   count_launch();
   FK_CUDA(cudaGetLastError());
   return FK_OK;

@@ -146,10 +146,24 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long w = (long long)blockIdx.x * kWarpsPerBlock + warp;
   float my_max = 0.f;
-  if (w < (long long)B * K) {
+  const bool live = w < (long long)B * K;
+  int cnt = 0, off = 0;
+  if (FROM_PIECES) {
+    // launched dependent on the segment reduce (do_update): the counts and
+    // offsets come from the sort, two or more launches back, so they are
+    // complete once this grid runs and are read before the wait; the
+    // partial sums are read after it
+    if (live) {
+      cnt = __ldg(counts + w);
+      off = __ldg(offsets + w);
+    }
+    pdl_wait();
+    pdl_trigger();
+  } else if (live) {
+    cnt = __ldg(counts + w);
+  }
+  if (live) {
     const int b = (int)(w / K), k = (int)(w % K);
-    const int cnt = __ldg(counts + w);
-    const int off = FROM_PIECES ? __ldg(offsets + w) : 0;  // both loads in flight together
     int p0 = 0, pl = -1;
     if (FROM_PIECES && cnt > 0) {
       p0 = off / kPiece;
@@ -308,14 +322,17 @@ int fin_t(const float *sums, const float *first, int pieces, const int32_t *coun
           const int32_t *offsets, float *centers, void *ch, void *cnx, int B, int K, int d,
           long long Kpad, unsigned *maxshift, int *err, cudaStream_t s) {
   const unsigned g = blocks_for((long long)B * K);
-  if (d % 4 == 0)
-    k_finalize<T, true, FP><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, centers,
-                                                              (T *)ch, (T *)cnx, B, K, d, Kpad, maxshift, err);
-  else
-    k_finalize<T, false, FP><<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, centers,
-                                                               (T *)ch, (T *)cnx, B, K, d, Kpad, maxshift, err);
+  // from pieces (do_update): a dependent launch after the segment reduce
+  auto go = [&](auto kern) -> cudaError_t {
+    if (FP)
+      return launch_pdl(kern, dim3(g), dim3(kWarpsPerBlock * 32), 0, s, sums, first, pieces, counts, offsets,
+                        centers, (T *)ch, (T *)cnx, B, K, d, Kpad, maxshift, err);
+    kern<<<g, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, centers, (T *)ch, (T *)cnx, B,
+                                           K, d, Kpad, maxshift, err);
+    return cudaGetLastError();
+  };
+  FK_CUDA(d % 4 == 0 ? go(k_finalize<T, true, FP>) : go(k_finalize<T, false, FP>));
   count_launch();
-  FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
 

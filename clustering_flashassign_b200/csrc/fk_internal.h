@@ -98,6 +98,33 @@ const char *last_error();
 size_t esize(int dtype);
 int num_sms();
 
+// Programmatic dependent launch: the kernels of one Lloyd iteration are
+// launched so that each may start while its predecessor in the stream drains.
+// A kernel launched this way calls pdl_wait() before it reads anything an
+// earlier kernel of the stream writes (or writes anything an earlier kernel
+// still reads), and pdl_trigger() only after its own pdl_wait(), so a kernel
+// that has started implies that every kernel two or more launches back has
+// completed.  After a memset or a copy the launch is ordinary.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---- kernels (launchers return fk_status) ----
 // Centroid preparation for the tensor-core assign: cnx[b, k, 0..15] = the
 // extension row of centroid k (digits of ||c||^2 / 2, see fk_norms.cuh), zero

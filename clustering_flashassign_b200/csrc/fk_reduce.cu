@@ -62,6 +62,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_segreduce(const T *__restrict__
                                                            float *__restrict__ first) {
   const int lane = threadIdx.x & 31;
   const long long item = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_trigger();
   if (item >= items) return;
   const int cb = (int)(item % colblocks);
   const long long rest = item / colblocks;
@@ -210,6 +212,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_segreduce16(const T *__restrict
   extern __shared__ __align__(16) uint8_t red_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long item = (long long)blockIdx.x * kWarps + warp;
+  pdl_wait();
+  pdl_trigger();
   if (item >= items) return;
   const int cb = (int)(item % colblocks);
   const long long rest = item / colblocks;
@@ -317,10 +321,9 @@ int launch16(const void *x, const int2 *kv, int B, int N, int K, int d, float *s
   const int colblocks = (d + 127) / 128;
   const long long items = (long long)B * pieces * colblocks;
   const unsigned grid = (unsigned)((items + kWarps - 1) / kWarps);
-  k_segreduce16<T><<<grid, kWarps * 32, shm, s>>>((const T *)x, kv, N, K, d, pieces, colblocks, items,
-                                                  sums, first);
+  FK_CUDA(launch_pdl(k_segreduce16<T>, dim3(grid), dim3(kWarps * 32), shm, s, (const T *)x, kv, N, K, d,
+                     pieces, colblocks, items, sums, first));
   count_launch();
-  FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
 
@@ -331,10 +334,9 @@ int launch(const void *x, const int2 *kv, int B, int N, int K, int d, float *sum
   const int colblocks = (d + 32 * VEC - 1) / (32 * VEC);
   const long long items = (long long)B * pieces * colblocks;
   const unsigned grid = (unsigned)((items + kWarps - 1) / kWarps);
-  k_segreduce<T, VEC><<<grid, kWarps * 32, 0, s>>>((const T *)x, kv, N, K, d, pieces, colblocks,
-                                                   items, sums, first);
+  FK_CUDA(launch_pdl(k_segreduce<T, VEC>, dim3(grid), dim3(kWarps * 32), 0, s, (const T *)x, kv, N, K, d,
+                     pieces, colblocks, items, sums, first));
   count_launch();
-  FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
 

@@ -127,7 +127,7 @@ __device__ __forceinline__ void tile_bases(const int32_t *counts, const uint32_t
   uint32_t local = 0;
   for (int bin = lo; bin < hi; ++bin) {
     local += (uint32_t)__ldg(counts + bin);
-    out[bin] = __ldg(gb + bin);
+    out[bin] = gb[bin];  // a plain load: the scatter may zero this row afterwards
   }
   uint32_t incl = local;
 #pragma unroll
@@ -184,9 +184,15 @@ __global__ void __launch_bounds__(kSortThreads) k_tile_hist(const int32_t *__res
 //   H[b][t][bin] <- sum over tiles t' < t of the bin (in place),
 //   counts[b][bin] = the bin's total.
 __global__ void __launch_bounds__(kSortThreads) k_scan_tiles(uint32_t *__restrict__ H, int bins,
-                                                             int T, int32_t *__restrict__ counts) {
+                                                             int T, int32_t *__restrict__ counts,
+                                                             unsigned *__restrict__ zero_word) {
   __shared__ uint32_t part[kSortWarps][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
+  // the update's max-shift word, zeroed here rather than by a memset that
+  // would break the chain of dependent launches
+  if (zero_word && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *zero_word = 0u;
   const int b = blockIdx.y, bin = blockIdx.x * 32 + lane;
   const bool on = bin < bins;
   const int per = (T + kSortWarps - 1) / kSortWarps;
@@ -224,12 +230,13 @@ __global__ void __launch_bounds__(kSortThreads) k_scan_tiles(uint32_t *__restric
 // It writes vals_out[pos] = vals_in ? vals_in[i] : i and keys_out[pos] = key
 // (each when not NULL), or the pair kv_out[pos] = (key, value): one 8-byte
 // store per point where the update needs both.  The CTA of tile 0 also writes
-// offsets_out[b] (when not NULL).
+// offsets_out[b] (when not NULL).  zero_g: the tile's row of G is zeroed once
+// read, so a histogram that the assign accumulates starts from zero again.
 __global__ void __launch_bounds__(kSortThreads) k_tile_scatter(
     const int32_t *__restrict__ keys, const int32_t *__restrict__ vals_in, int N, int K, int T,
-    PassCfg pc, const uint32_t *__restrict__ G, const int32_t *__restrict__ counts,
+    PassCfg pc, uint32_t *__restrict__ G, const int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets_out, int32_t *__restrict__ keys_out,
-    int32_t *__restrict__ vals_out, int2 *__restrict__ kv_out, int *err) {
+    int32_t *__restrict__ vals_out, int2 *__restrict__ kv_out, int zero_g, int *err) {
   extern __shared__ uint32_t sm[];  // base[bins], cnt[kSortWarps][bins]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, b = blockIdx.y;
@@ -237,6 +244,9 @@ __global__ void __launch_bounds__(kSortThreads) k_tile_scatter(
   uint32_t *tb = sm;
   uint32_t *cnt_all = sm + bins;
   const long long base = (long long)tile * kSortTile + warp * kWarpPoints;
+  for (int e = threadIdx.x; e < kSortWarps * bins; e += kSortThreads) cnt_all[e] = 0;
+  pdl_wait();
+  pdl_trigger();
   // the keys (and values) are fetched first; their latency overlaps the scan
   WarpKeys wk;
   fetch_warp_keys(wk, keys + (size_t)b * N, base, N, lane);
@@ -248,8 +258,10 @@ __global__ void __launch_bounds__(kSortThreads) k_tile_scatter(
       vals[r] = i < N ? __ldg(vals_in + (size_t)b * N + i) : 0;
     }
   }
-  for (int e = threadIdx.x; e < kSortWarps * bins; e += kSortThreads) cnt_all[e] = 0;
-  tile_bases(counts + (size_t)b * bins, G + ((size_t)b * T + tile) * bins, bins, tb);
+  uint32_t *grow = G + ((size_t)b * T + tile) * bins;
+  tile_bases(counts + (size_t)b * bins, grow, bins, tb);  // ends with __syncthreads
+  if (zero_g)
+    for (int bin = threadIdx.x; bin < bins; bin += kSortThreads) grow[bin] = 0u;
   if (tile == 0 && offsets_out)  // tile 0's prefix is zero: its bases are the offsets
     for (int bin = threadIdx.x; bin < bins; bin += kSortThreads)
       offsets_out[(size_t)b * bins + bin] = (int32_t)tb[bin];
@@ -382,15 +394,13 @@ int one_pass(Workspace *ws, const int32_t *keys_in, const int32_t *vals_in, int 
     count_launch();
     FK_CUDA(cudaGetLastError());
   }
-  k_scan_tiles<<<dim3((unsigned)((pc.bins + 31) / 32), (unsigned)B), kSortThreads, 0, s>>>(
-      H, pc.bins, T, digit_counts);
+  FK_CUDA(launch_pdl(k_scan_tiles, dim3((unsigned)((pc.bins + 31) / 32), (unsigned)B), dim3(kSortThreads),
+                    0, s, H, pc.bins, T, digit_counts, ws->maxshift));
   count_launch();
-  FK_CUDA(cudaGetLastError());
-  k_tile_scatter<<<grid, kSortThreads, shm_s, s>>>(keys_in, vals_in, N, K, T, pc, H, digit_counts,
-                                                   offsets_out, keys_out, vals_out, kv_out,
-                                                   ws->err);
+  FK_CUDA(launch_pdl(k_tile_scatter, grid, dim3(kSortThreads), shm_s, s, keys_in, vals_in, N, K, T, pc, H,
+                     (const int32_t *)digit_counts, offsets_out, keys_out, vals_out, kv_out,
+                     have_hist ? 1 : 0, ws->err));
   count_launch();
-  FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
 
