@@ -116,8 +116,12 @@ int assign_f32_tc(Workspace *ws, const float *x, const float *c, const float *x3
   FK_TRY(launch_split3(c, (long long)B * K, d, (float *)ws->c3.p, true, s));
   FK_TRY(ensure(ws->cn, ext_bytes(B, Kpad)));
   FK_TRY(launch_prep_ext_f32(c, B, K, d, Kpad, ws->cn.p, s));
+  // the widened point tiles (128 x 3d x 4 bytes) do not stay in L2 across a
+  // tile's chunks: one work item per (tile, chunk), consecutive CTAs sharing a
+  // tile's reads, merged through per-point keys
+  FK_TRY(ensure_zeroed(ws->keys64, (size_t)B * N * sizeof(unsigned long long), s));
   return launch_assign_tc(x3, ws->c3.p, ws->cn.p, nullptr, FK_F32, B, N, K, d3, Kpad, ids, ws->err, s,
-                          hist);
+                          hist, (unsigned long long *)ws->keys64.p);
 }
 
 int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const void *cnx,
@@ -130,6 +134,8 @@ int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const void
       return assign_f32_tc(ws, (const float *)x, (const float *)cdt, x3, B, N, K, d, Kpad, ids, s, hist);
     return launch_assign_f32((const float *)x, (const float *)cdt, B, N, K, d, ids, s);
   }
+  // 16-bit split-d tiles (128 x d x 2 bytes) stay in L2 across a tile's
+  // chunks, so one work item per tile (no per-chunk merge) is the faster order
   return launch_assign_tc(x, cdt, cnx, xn, dtype, B, N, K, d, Kpad, ids, ws->err, s, hist);
 }
 

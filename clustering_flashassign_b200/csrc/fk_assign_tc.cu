@@ -80,7 +80,18 @@ struct TcArgs {
   // optional: the counting sort's tile histogram, H[b][row / 2048][id] += 1
   uint32_t *hist;
   int hist_tiles;
+  // split-d only, optional: per-point packed (value, index) keys; then every
+  // (tile, chunk) pair is its own work item and chunks merge by atomicMax
+  unsigned long long *keys;
 };
+
+// (value, index) as one 64-bit key whose unsigned order is: larger value
+// first, then lower index (the value bits mapped to an order-preserving uint).
+__device__ __forceinline__ unsigned long long pack_argmax(float v, int idx) {
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)o << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)idx);
+}
 
 template <bool RESIDENT, int KB, int STAGES>
 struct Layout {
@@ -301,6 +312,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the set-up above overlaps the previous kernel of the stream; everything
   // below may read what it wrote
   pdl_wait();
+  // Work items: a point tile with all its chunks, or (split-d with keys) one
+  // (tile, chunk) pair, consecutive CTAs taking consecutive chunks of one tile
+  // so that they read its K-blocks at about the same time (shared in L2).
+  const bool per_chunk = !RESIDENT && a.keys != nullptr;
+  const int ntask = per_chunk ? a.total_tiles * a.nchunks : a.total_tiles;
+  auto task_tile = [&](int t) { return per_chunk ? t / a.nchunks : t; };
+  auto chunk_lo = [&](int t) { return per_chunk ? t % a.nchunks : 0; };
+  auto chunk_hi = [&](int t) { return per_chunk ? t % a.nchunks + 1 : a.nchunks; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -323,10 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       if (RESIDENT && (int)blockIdx.x < a.total_tiles) ok = load_x(blockIdx.x);
-      for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x) {
+      for (int task = blockIdx.x; ok && task < ntask; task += gridDim.x) {
+        const int tile = task_tile(task);
         const int b = tile / a.tiles_per_batch;
         const int row0 = (tile % a.tiles_per_batch) * kTileM;
-        for (int c = 0; ok && c < a.nchunks; ++c) {
+        for (int c = chunk_lo(task); ok && c < chunk_hi(task); ++c) {
           if (RESIDENT) {  // the whole chunk and its norm rows in one stage
             const int s = f % STAGES;
             if (!mbar_wait(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
@@ -373,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t f = 0, g = 0, h = 0, e = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x) {
+      for (int task = blockIdx.x; ok && task < ntask; task += gridDim.x) {
         int xb = 0;
         if (RESIDENT) {
           xb = g & 1;
@@ -381,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
         }
         const uint32_t a_ext = aext_base + (RESIDENT ? xb * kAExtBytes : 0u);
-        for (int c = 0; ok && c < a.nchunks; ++c) {
+        for (int c = chunk_lo(task); ok && c < chunk_hi(task); ++c) {
           const int ab = h & 1;
           if (!mbar_wait(accempty(ab), ((h >> 1) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
@@ -519,12 +539,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 32; ++i) colb[i] = 0x03020100u + 0x04040404u * i;
     uint32_t h = 0, u = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x, ++u) {
+    for (int task = blockIdx.x; ok && task < ntask; task += gridDim.x, ++u) {
+      const int tile = task_tile(task);
       const int b = tile / a.tiles_per_batch;
       const int row0 = (tile % a.tiles_per_batch) * kTileM;
       float best = __int_as_float(0xff800000);  // -inf
       int bidx = 0;                              // chunk (packed) or column (exact) of best
-      for (int c = 0; c < a.nchunks; ++c, ++h) {
+      for (int c = chunk_lo(task); c < chunk_hi(task); ++c, ++h) {
         const int ab = h & 1;
         if (!warp_wait(accfull(ab), (h >> 1) & 1, abort_flag, a.err, lane)) { ok = false; break; }
         tc_fence_after();
@@ -604,9 +625,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(mempty(p));
         const float ov = o.x;
         const int oi = __float_as_int(o.y);
-        if (ov > val || (ov == val && oi < idx)) idx = oi;
+        if (ov > val || (ov == val && oi < idx)) {  // the value travels too: the keys compare it
+          val = ov;
+          idx = oi;
+        }
         const int row = row0 + r_in_tile;
-        if (row < a.N) {
+        if (row < a.N && per_chunk) {  // this chunk's best; the chunks merge in the keys
+          atomicMax(a.keys + (size_t)b * a.N + row, pack_argmax(val, idx));
+        } else if (row < a.N) {
           a.ids[(size_t)b * a.N + row] = idx;
           if (a.hist)  // the sort's first kernel, fused: count the id in its sort tile
             atomicAdd(a.hist + ((size_t)b * a.hist_tiles + row / kSortTile) * a.K + idx, 1u);
@@ -619,6 +645,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Split-d with per-chunk work items: ids from the merged keys (and the
+// sort's tile histogram, when fused), then the keys are cleared for the next
+// launch.
+__global__ void __launch_bounds__(256)
+    k_keys_to_ids(unsigned long long *__restrict__ keys, long long n, int N, int K,
+                  int32_t *__restrict__ ids, uint32_t *__restrict__ hist, int hist_tiles) {
+  pdl_wait();
+  for (long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x; r < n;
+       r += (long long)gridDim.x * blockDim.x) {
+    const unsigned long long key = keys[r];
+    const int idx = (int)(0xFFFFFFFFu - (uint32_t)key);
+    // every point gets a key from every chunk unless the assign gave up (its
+    // timeout is in the device error word): then write 0 and count nothing
+    const bool valid = key != 0ull && (unsigned)idx < (unsigned)K;
+    ids[r] = valid ? idx : 0;
+    if (hist && valid) {
+      const long long b = r / N;
+      const int row = (int)(r - b * N);
+      atomicAdd(hist + ((size_t)b * hist_tiles + row / kSortTile) * K + idx, 1u);
+    }
+    keys[r] = 0ull;
   }
 }
 
@@ -735,7 +785,7 @@ int launch_point_norms(const void *x, int dtype, long long rows, int d, float *x
 
 int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float *xn, int dtype,
                      int B, long long N, int K, int d, long long Kpad, int32_t *ids, int *err,
-                     cudaStream_t s, uint32_t *hist) {
+                     cudaStream_t s, uint32_t *hist, unsigned long long *keys) {
   // K-blocks are 128-byte rows: 64 16-bit elements or 32 fp32 (read as tf32);
   // norm rows are 32 bytes: 16 or 8 elements
   const int blk = dtype == FK_F32 ? 32 : kBlockK;
@@ -759,11 +809,25 @@ int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float
   a.ids = ids;
   a.err = err;
   a.idesc = sm100::idesc_f32acc(dtype == FK_F32 ? 2u : dtype == FK_BF16 ? 1u : 0u, kTileM, kChunkN);
+  // split-d (fp32, or more than two 16-bit K-blocks): with keys, one work item
+  // per (tile, chunk) and a merge of the chunks' results
+  const bool splitd = dtype == FK_F32 || a.kblocks > 2;
+  a.keys = (splitd && keys && total * a.nchunks <= 0x7fffffffLL) ? keys : nullptr;
+  if (a.keys) a.hist = nullptr;  // counted when the ids are written
+  const long long tasks = a.keys ? total * a.nchunks : total;
   int grid = num_sms();
-  if (total < grid) grid = (int)total;
-  if (dtype == FK_F32) return launch_typed<float>(tmx, tmc, tme, a, grid, s);
-  if (dtype == FK_BF16) return launch_typed<__nv_bfloat16>(tmx, tmc, tme, a, grid, s);
-  return launch_typed<__half>(tmx, tmc, tme, a, grid, s);
+  if (tasks < grid) grid = (int)tasks;
+  if (dtype == FK_F32) FK_TRY(launch_typed<float>(tmx, tmc, tme, a, grid, s));
+  else if (dtype == FK_BF16) FK_TRY(launch_typed<__nv_bfloat16>(tmx, tmc, tme, a, grid, s));
+  else FK_TRY(launch_typed<__half>(tmx, tmc, tme, a, grid, s));
+  if (!a.keys) return FK_OK;
+  const long long n = (long long)B * N;
+  long long blocks = (n + 255) / 256;
+  if (blocks > (long long)num_sms() * 8) blocks = (long long)num_sms() * 8;
+  FK_CUDA(launch_pdl(k_keys_to_ids, dim3((unsigned)blocks), dim3(256), 0, s, keys, n, (int)N, K, ids, hist,
+                     a.hist_tiles));
+  count_launch();
+  return FK_OK;
 }
 
 }  // namespace fk

@@ -55,6 +55,7 @@ struct Workspace {
   DevBuf cn, ch, sums, first, counts, offsets, table, digit_off, kv, keys_b, vals_b;
   DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2], gsum, gcounts, xn, ids_alt;
   DevBuf x3, c3;                  // 3xTF32 operands of the fp32 tensor-core assign
+  DevBuf keys64;                  // split-d per-point argmax keys, kept zeroed
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
   cudaEvent_t shift_ev = nullptr;  // the max-shift copy of the Lloyd loop has landed
@@ -76,6 +77,7 @@ int cuda_status(cudaError_t e, const char *what);
   } while (0)
 
 int ensure(DevBuf &b, size_t bytes);               // grow-only device buffer
+int ensure_zeroed(DevBuf &b, size_t bytes, cudaStream_t s);  // zero-filled when (re)allocated
 int workspace_for(cudaStream_t s, Workspace **out);
 
 // Launch accounting and event timing.
@@ -165,7 +167,9 @@ int launch_prep_ext_f32(const float *c, int B, int K, int d, long long Kpad, voi
 // (run_sort_prehist then skips its histogram kernel).
 int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float *xn, int dtype,
                      int B, long long N, int K, int d, long long Kpad, int32_t *ids, int *err,
-                     cudaStream_t s, uint32_t *hist = nullptr);
+                     cudaStream_t s, uint32_t *hist = nullptr, unsigned long long *keys = nullptr);
+// keys: (B, N) zeroed scratch for the split-d variant's per-chunk work items
+// (left zeroed again); NULL keeps one work item per point tile.
 // xn[r] = ||x_r||^2 (fp32 accumulation) for `rows` rows of d 16-bit elements.
 int launch_point_norms(const void *x, int dtype, long long rows, int d, float *xn, cudaStream_t s);
 

@@ -39,6 +39,13 @@ int cuda_status(cudaError_t e, const char *what) {
   return FK_ECUDA;
 }
 
+int ensure_zeroed(DevBuf &b, size_t bytes, cudaStream_t s) {
+  const size_t had = b.bytes;  // a new allocation always changes the size (it only grows)
+  FK_TRY(ensure(b, bytes));
+  if (b.bytes != had) FK_CUDA(cudaMemsetAsync(b.p, 0, b.bytes, s));
+  return FK_OK;
+}
+
 int ensure(DevBuf &b, size_t bytes) {
   if (bytes == 0) bytes = 16;
   if (b.bytes >= bytes) return FK_OK;
@@ -107,7 +114,7 @@ int release_device_workspaces() {
     }
     Workspace *ws = it->second;
     DevBuf *bufs[] = {&ws->cn, &ws->ch, &ws->sums, &ws->first, &ws->counts, &ws->offsets,
-                      &ws->table, &ws->digit_off, &ws->kv, &ws->x3, &ws->c3, &ws->keys_b,
+                      &ws->table, &ws->digit_off, &ws->kv, &ws->x3, &ws->c3, &ws->keys64, &ws->keys_b,
                       &ws->vals_b, &ws->xres, &ws->init_dev, &ws->ids_dev, &ws->centers_dev,
                       &ws->chunk[0], &ws->chunk[1], &ws->gsum, &ws->gcounts, &ws->xn, &ws->ids_alt};
     for (DevBuf *b : bufs) free_buf(*b);
