@@ -153,9 +153,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     // offsets come from the sort, two or more launches back, so they are
     // complete once this grid runs and are read before the wait; the
     // partial sums are read after it
-    if (live) {
-      cnt = __ldg(counts + w);
-      off = __ldg(offsets + w);
+    if (live) {  // through L2 (.cg): no reliance on this SM's L1 holding nothing stale
+      cnt = __ldcg(counts + w);
+      off = __ldcg(offsets + w);
     }
     pdl_wait();
     pdl_trigger();
