@@ -1,4 +1,5 @@
-// FlashAssign on sm_100a tensor cores (step a1 for fp16 / bf16 inputs).
+// FlashAssign on sm_100a tensor cores (step a1 for fp16 / bf16 inputs, and
+// for fp32 inputs as 3xTF32 on extended rows built by fk_tf32.cu).
 //
 // ids[b,i] = argmin_k ||x_i - c_k||^2, fp32 accumulation, lowest k on ties,
 // without ever writing the (B, N, K) distance matrix ("Flash-KMeans: Fast and
@@ -42,7 +43,13 @@
 //               fallback").  acc = x.c - ||c||^2 / 2 and the epilogue keeps an
 //               exact (value, column) argmax; its cost is spread over d / 64
 //               K-blocks.  The threshold is set by the shared-memory budget of
-//               this design, not the pages' 512.
+//               this design, not the pages' 512.  Instantiated for fp32
+//               elements too (kind::tf32, K = 8 per MMA: a 128-byte K-block row
+//               holds 32 values, so layouts and stage sizes are unchanged).
+//               With a keys buffer every (tile, chunk) pair is its own work
+//               item, consecutive CTAs taking one tile's chunks so they share
+//               its reads in L2; the chunks merge by a 64-bit atomicMax per
+//               point and k_keys_to_ids writes the ids.
 // Rows past N and centroid rows past K are zero-filled by TMA; padded centroid
 // columns carry a sentinel norm row (acc about -2^31 or below) so they never win.
 #include <cuda.h>
