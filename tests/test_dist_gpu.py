@@ -95,7 +95,8 @@ def _dp(xd, cd, iters, steps=None):
     return ids, cen
 
 
-@pytest.mark.parametrize("dtype,d", [("f16", 128), ("bf16", 64), ("f32", 32), ("f16", 256)])
+@pytest.mark.parametrize("dtype,d", [("f16", 128), ("bf16", 64), ("f32", 32), ("f16", 256),
+                                     ("f32", 128)])   # fp32 on the tensor cores (K * d >= 16384)
 def test_one_rank_is_fk_lloyd(dtype, d):
     B, N, K = 2, 4000, 200
     x, _, c = case(B, N, K, d, dtype, seed=37)
