@@ -32,13 +32,14 @@ LIB_PATH = os.path.join(_HERE, "libfk.so")
 FK_F32, FK_F16, FK_BF16 = 0, 1, 2
 FK_OK, FK_EINVAL, FK_ENOMEM, FK_ECUDA, FK_ETIMEOUT, FK_EUNSUPPORTED = range(6)
 FK_HOST_AUTO, FK_HOST_RESIDENT, FK_HOST_STREAM = 0, 1, 2
+FK_FAULT_NONE, FK_FAULT_ALLOC, FK_FAULT_H2D, FK_FAULT_LAUNCH = 0, 1, 2, 3
 
 DTYPES = {torch.float32: FK_F32, torch.float16: FK_F16, torch.bfloat16: FK_BF16}
 
 EXPORTS = ["fk_assign", "fk_update", "fk_sort", "fk_lloyd", "fk_assign_noalloc", "fk_status_string",
            "fk_last_error", "fk_device_error", "fk_release", "fk_profile_enable", "fk_profile_read",
            "fk_launch_count", "fk_version", "fk_selftest_bounded_wait", "fk_point_norms",
-           "fk_init_centers", "fk_lloyd_step_partial", "fk_update_finalize"]
+           "fk_init_centers", "fk_lloyd_step_partial", "fk_update_finalize", "fk_inject_fault"]
 
 
 class FkError(RuntimeError):
@@ -90,6 +91,7 @@ def _load():
         "fk_lloyd_step_partial": (I, [ctypes.POINTER(FkShape), P, P, P, P, P, P, P,
                                       ctypes.POINTER(FkOptions)]),
         "fk_update_finalize": (I, [P, P, I, I, I, I, P, P, P, P]),
+        "fk_inject_fault": (I, [I, LL]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -228,6 +230,12 @@ def fk_device_error(stream=None) -> int:
 def fk_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
     """Status of a kernel whose mbarrier wait can never complete (FK_ETIMEOUT expected)."""
     return int(lib.fk_selftest_bounded_wait(ctypes.c_longlong(int(limit_ns)), _stream(stream)))
+
+
+def fk_inject_fault(kind: int, nth: int = 1) -> None:
+    """Arm one host-side failure (FK_FAULT_ALLOC / _H2D / _LAUNCH) at its nth occurrence;
+    FK_FAULT_NONE disarms.  For tests of the error paths; no GPU is faulted."""
+    _check(lib.fk_inject_fault(int(kind), int(nth)), "fk_inject_fault")
 
 
 def fk_release() -> None:

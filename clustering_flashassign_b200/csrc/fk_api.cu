@@ -196,6 +196,7 @@ int streamed_pass(Workspace *ws, const fk_shape &sh, const char *xh, long long c
       const long long nc = (n0 + chunk <= N) ? chunk : N - n0;
       void *xb = ws->chunk[buf].p;
       FK_CUDA(cudaStreamWaitEvent(ws->copy_stream, ws->freed[buf], 0));
+      if (fault_hit(FK_FAULT_H2D)) return set_error(FK_ECUDA, "injected host-to-device copy failure (FK_FAULT)");
       FK_CUDA(cudaMemcpyAsync(xb, xh + ((size_t)b * N + n0) * d * es, (size_t)nc * d * es,
                               cudaMemcpyHostToDevice, ws->copy_stream));
       FK_CUDA(cudaEventRecord(ws->ready[buf], ws->copy_stream));
@@ -464,6 +465,7 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
   const void *init_dev = init_centers;
   if (li != LOC_DEVICE) {
     FK_TRY(ensure(ws->init_dev, cbytes));
+    if (fault_hit(FK_FAULT_H2D)) return set_error(FK_ECUDA, "injected host-to-device copy failure (FK_FAULT)");
     FK_CUDA(cudaMemcpyAsync(ws->init_dev.p, init_centers, cbytes, cudaMemcpyHostToDevice, s));
     init_dev = ws->init_dev.p;
   }
@@ -494,6 +496,7 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
                             &iters, o.chunk_points, o.verbose));
     } else {
       FK_TRY(ensure(ws->xres, xbytes));
+      if (fault_hit(FK_FAULT_H2D)) return set_error(FK_ECUDA, "injected host-to-device copy failure (FK_FAULT)");
       FK_CUDA(cudaMemcpyAsync(ws->xres.p, x, xbytes, cudaMemcpyHostToDevice, s));
       xdev = ws->xres.p;
     }
@@ -618,5 +621,7 @@ int fk_profile_read(fk_profile *out, int reset) { return profile_read(out, reset
 long long fk_launch_count(void) { return launch_count(); }
 
 int fk_version(void) { return 100; }
+
+int fk_inject_fault(int kind, long long nth) { return set_fault(kind, nth); }
 
 }  // extern "C"

@@ -68,7 +68,7 @@ int launch_assign_f32(const float *x, const float *c, int B, long long N, int K,
                       int32_t *ids, cudaStream_t s) {
   dim3 grid((unsigned)((N + kThreads - 1) / kThreads), (unsigned)B);
   k_assign_f32<<<grid, kThreads, 0, s>>>(x, c, (int)N, K, d, ids);
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }

@@ -708,7 +708,7 @@ int point_norms_t(const void *x, long long rows, int d, float *xn, cudaStream_t 
   const long long cap = (long long)num_sms() * 16;
   if (blocks > cap) blocks = cap;
   k_point_norms<T><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const T *>(x), rows, d, xn);
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
@@ -767,7 +767,7 @@ int launch_variant(const CUtensorMap &tmx, const CUtensorMap &tmc, const CUtenso
   }
   FK_CUDA(launch_pdl(k_flash_assign<T, RESIDENT, KB, STAGES>, dim3(grid), dim3(kThreads), L::kAlloc, s, tmx, tmc,
                      tme, a));
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
@@ -833,7 +833,7 @@ int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float
   if (blocks > (long long)num_sms() * 8) blocks = (long long)num_sms() * 8;
   FK_CUDA(launch_pdl(k_keys_to_ids, dim3((unsigned)blocks), dim3(256), 0, s, keys, n, (int)N, K, ids, hist,
                      a.hist_tiles));
-  count_launch();
+  FK_TRY(launched());
   return FK_OK;
 }
 

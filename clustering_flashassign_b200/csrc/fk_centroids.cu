@@ -299,7 +299,7 @@ int prep_t(const void *c, int B, int K, int d, long long Kpad, void *cnx, int *e
   const unsigned g = blocks_for((long long)B * Kpad);
   if (d % 4 == 0) k_prep_cn<T, true><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)c, B, K, d, Kpad, (T *)cnx, err);
   else k_prep_cn<T, false><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)c, B, K, d, Kpad, (T *)cnx, err);
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
@@ -312,7 +312,7 @@ int init_t(const void *init, int B, int K, int d, long long Kpad, float *master,
     k_init<T, true><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)init, B, K, d, Kpad, master, (T *)ch, (T *)cnx, err);
   else
     k_init<T, false><<<g, kWarpsPerBlock * 32, 0, s>>>((const T *)init, B, K, d, Kpad, master, (T *)ch, (T *)cnx, err);
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
@@ -332,7 +332,7 @@ int fin_t(const float *sums, const float *first, int pieces, const int32_t *coun
     return cudaGetLastError();
   };
   FK_CUDA(d % 4 == 0 ? go(k_finalize<T, true, FP>) : go(k_finalize<T, false, FP>));
-  count_launch();
+  FK_TRY(launched());
   return FK_OK;
 }
 
@@ -379,7 +379,7 @@ int launch_accumulate(const float *sums, const float *first, int pieces, const i
   else
     k_accumulate<false><<<grid, kWarpsPerBlock * 32, 0, s>>>(sums, first, pieces, counts, offsets, K, d, gsum,
                                                              gcounts, overwrite ? 1 : 0);
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }

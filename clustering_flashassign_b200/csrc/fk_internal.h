@@ -81,7 +81,12 @@ int ensure_zeroed(DevBuf &b, size_t bytes, cudaStream_t s);  // zero-filled when
 int workspace_for(cudaStream_t s, Workspace **out);
 
 // Launch accounting and event timing.
-void count_launch(int n = 1);
+// Launch accounting; returns FK_ECUDA when an injected launch fault fires.
+int launched(int n = 1);
+// Host-side fault injection: true when the armed failure of `kind`
+// (FK_FAULT_ALLOC / _H2D / _LAUNCH) fires here.
+bool fault_hit(int kind);
+int set_fault(int kind, long long nth);
 enum Phase { PH_ASSIGN = 0, PH_SORT = 1, PH_REDUCE = 2, PH_FINALIZE = 3, PH_UPDATE = 4, PH_COUNT = 5 };
 struct PhaseTimer {
   cudaEvent_t a = nullptr, b = nullptr;

@@ -323,7 +323,7 @@ int launch16(const void *x, const int2 *kv, int B, int N, int K, int d, float *s
   const unsigned grid = (unsigned)((items + kWarps - 1) / kWarps);
   FK_CUDA(launch_pdl(k_segreduce16<T>, dim3(grid), dim3(kWarps * 32), shm, s, (const T *)x, kv, N, K, d,
                      pieces, colblocks, items, sums, first));
-  count_launch();
+  FK_TRY(launched());
   return FK_OK;
 }
 
@@ -336,7 +336,7 @@ int launch(const void *x, const int2 *kv, int B, int N, int K, int d, float *sum
   const unsigned grid = (unsigned)((items + kWarps - 1) / kWarps);
   FK_CUDA(launch_pdl(k_segreduce<T, VEC>, dim3(grid), dim3(kWarps * 32), 0, s, (const T *)x, kv, N, K, d,
                      pieces, colblocks, items, sums, first));
-  count_launch();
+  FK_TRY(launched());
   return FK_OK;
 }
 

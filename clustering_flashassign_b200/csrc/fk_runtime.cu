@@ -1,6 +1,7 @@
 // Runtime pieces of libfk: status text, per-(device, stream) workspaces,
 // launch accounting and event-based phase timing.
 #include <cstdio>
+#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -49,6 +50,8 @@ int ensure_zeroed(DevBuf &b, size_t bytes, cudaStream_t s) {
 int ensure(DevBuf &b, size_t bytes) {
   if (bytes == 0) bytes = 16;
   if (b.bytes >= bytes) return FK_OK;
+  if (fault_hit(FK_FAULT_ALLOC))
+    return set_error(FK_ENOMEM, "injected allocation failure (FK_FAULT)");
   if (b.p) {
     FK_CUDA(cudaFree(b.p));
     b.p = nullptr;
@@ -132,12 +135,62 @@ int release_device_workspaces() {
   return FK_OK;
 }
 
-void count_launch(int n) {
+// ---- host-side fault injection (tests of the error paths; no GPU is faulted)
+namespace {
+std::mutex g_fault_mu;
+std::atomic<int> g_fault_kind{-1};  // -1: FK_FAULT not read yet
+long long g_fault_left = 0;         // occurrences of the kind still to pass, the last fires
+
+int fault_kind_of(const std::string &name) {
+  if (name == "alloc") return FK_FAULT_ALLOC;
+  if (name == "h2d") return FK_FAULT_H2D;
+  if (name == "launch") return FK_FAULT_LAUNCH;
+  return FK_FAULT_NONE;
+}
+
+// FK_FAULT=alloc|h2d|launch[:n] arms one failure at the n-th occurrence (default 1).
+void read_fault_env() {
+  int kind = FK_FAULT_NONE;
+  long long nth = 1;
+  if (const char *e = getenv("FK_FAULT")) {
+    std::string v(e);
+    const size_t colon = v.find(':');
+    kind = fault_kind_of(v.substr(0, colon));
+    if (colon != std::string::npos) nth = atoll(v.c_str() + colon + 1);
+  }
+  g_fault_left = nth > 0 ? nth : 1;
+  g_fault_kind.store(kind);
+}
+}  // namespace
+
+bool fault_hit(int kind) {
+  int k = g_fault_kind.load(std::memory_order_relaxed);
+  if (k == FK_FAULT_NONE) return false;
+  std::lock_guard<std::mutex> lk(g_fault_mu);
+  if (g_fault_kind.load() < 0) read_fault_env();
+  if (g_fault_kind.load() != kind) return false;
+  if (--g_fault_left > 0) return false;
+  g_fault_kind.store(FK_FAULT_NONE);  // fires once
+  return true;
+}
+
+int set_fault(int kind, long long nth) {
+  if (kind < FK_FAULT_NONE || kind > FK_FAULT_LAUNCH || nth < 1)
+    return set_error(FK_EINVAL, "fault kind must be FK_FAULT_NONE..FK_FAULT_LAUNCH and nth >= 1");
+  std::lock_guard<std::mutex> lk(g_fault_mu);
+  g_fault_left = nth;
+  g_fault_kind.store(kind);
+  return FK_OK;
+}
+
+int launched(int n) {
   g_launches.fetch_add(n, std::memory_order_relaxed);
   if (g_prof_level) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     g_prof_launches += n;
   }
+  if (fault_hit(FK_FAULT_LAUNCH)) return set_error(FK_ECUDA, "injected launch failure (FK_FAULT)");
+  return FK_OK;
 }
 
 long long launch_count() { return g_launches.load(); }

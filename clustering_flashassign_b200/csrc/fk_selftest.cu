@@ -48,7 +48,7 @@ extern "C" int fk_selftest_bounded_wait(long long limit_ns, fk_stream_t stream) 
   Workspace *ws;
   FK_TRY(workspace_for(s, &ws));
   k_wait_selftest<<<1, 32, 0, s>>>((unsigned long long)limit_ns, ws->err);
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   return fk_device_error(stream);
 }

@@ -391,16 +391,16 @@ int one_pass(Workspace *ws, const int32_t *keys_in, const int32_t *vals_in, int 
   const size_t shm_s = (size_t)(kSortWarps + 1) * pc.bins * sizeof(uint32_t);
   if (!have_hist) {
     k_tile_hist<<<grid, kSortThreads, shm_h, s>>>(keys_in, N, K, T, pc, H, ws->err);
-    count_launch();
+    FK_TRY(launched());
     FK_CUDA(cudaGetLastError());
   }
   FK_CUDA(launch_pdl(k_scan_tiles, dim3((unsigned)((pc.bins + 31) / 32), (unsigned)B), dim3(kSortThreads),
                     0, s, H, pc.bins, T, digit_counts, ws->maxshift));
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(launch_pdl(k_tile_scatter, grid, dim3(kSortThreads), shm_s, s, keys_in, vals_in, N, K, T, pc, H,
                      (const int32_t *)digit_counts, offsets_out, keys_out, vals_out, kv_out,
                      have_hist ? 1 : 0, ws->err));
-  count_launch();
+  FK_TRY(launched());
   return FK_OK;
 }
 
@@ -467,11 +467,11 @@ int run_sort(Workspace *ws, const int32_t *ids, int B, long long N_, int K, int3
   FK_CUDA(cudaMemsetAsync(cnt, 0, (size_t)B * K * sizeof(int32_t), s));
   const int use_smem = (size_t)K * 4 <= 64 * 1024 ? 1 : 0;
   k_count<<<dim3((unsigned)T, (unsigned)B), 256, use_smem ? K * 4 : 0, s>>>(ids, N, K, cnt, use_smem);
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   if (offsets) {
     k_offsets<<<B, 1024, 0, s>>>(cnt, K, offsets);
-    count_launch();
+    FK_TRY(launched());
     FK_CUDA(cudaGetLastError());
   }
   return FK_OK;

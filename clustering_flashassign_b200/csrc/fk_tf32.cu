@@ -70,7 +70,7 @@ int launch_split3(const float *src, long long rows, int d, float *dst, bool cent
   if (blocks == 0) return FK_OK;
   k_split3<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4 *>(src), rows, d / 4,
                                             reinterpret_cast<float4 *>(dst), centroids ? 1 : 0);
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
@@ -78,7 +78,7 @@ int launch_split3(const float *src, long long rows, int d, float *dst, bool cent
 int launch_prep_ext_f32(const float *c, int B, int K, int d, long long Kpad, void *cnx, cudaStream_t s) {
   const long long warps = (long long)B * Kpad;
   k_prep_ext_f32<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(c, B, K, d, Kpad, static_cast<float4 *>(cnx));
-  count_launch();
+  FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }

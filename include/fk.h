@@ -291,6 +291,23 @@ int fk_device_error(fk_stream_t stream);
  */
 int fk_selftest_bounded_wait(long long limit_ns, fk_stream_t stream);
 
+/*
+ * fk_inject_fault -- host-side fault injection for tests of the error paths
+ * (an interface addition; the pages have no counterpart).  Arms one failure
+ * that fires once, at the nth occurrence of its kind, without faulting any
+ * GPU:
+ *   FK_FAULT_ALLOC   a workspace allocation returns FK_ENOMEM,
+ *   FK_FAULT_H2D     a host-to-device copy of fk_lloyd (the resident upload,
+ *                    the initial centroids, a streamed chunk) returns FK_ECUDA
+ *                    before it is issued,
+ *   FK_FAULT_LAUNCH  the call that launched a kernel returns FK_ECUDA right
+ *                    after the launch (the kernel itself runs).
+ * FK_FAULT_NONE disarms.  The environment variable FK_FAULT=alloc|h2d|launch[:n]
+ * arms the same at the first check.  nth >= 1; FK_EINVAL otherwise.
+ */
+typedef enum { FK_FAULT_NONE = 0, FK_FAULT_ALLOC = 1, FK_FAULT_H2D = 2, FK_FAULT_LAUNCH = 3 } fk_fault;
+int fk_inject_fault(int kind, long long nth);
+
 /* Frees every workspace of the current device (no call may be in flight). */
 int fk_release(void);
 

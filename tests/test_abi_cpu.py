@@ -112,3 +112,12 @@ def test_data_parallel_pieces_validate_on_the_host():
     assert "counts is NULL" in fk.fk_last_error()
     assert L.fk_update_finalize(p, p, 1, 4, 8, 9, p, p, None, None) == fk.FK_EINVAL
     assert "unknown dtype" in fk.fk_last_error()
+
+
+def test_fault_injection_arguments():
+    import clustering_flashassign_b200 as fk
+    L = fk.lib
+    assert L.fk_inject_fault(7, 1) == fk.FK_EINVAL
+    assert L.fk_inject_fault(fk.FK_FAULT_ALLOC, 0) == fk.FK_EINVAL
+    assert L.fk_inject_fault(fk.FK_FAULT_ALLOC, 3) == fk.FK_OK
+    assert L.fk_inject_fault(fk.FK_FAULT_NONE, 1) == fk.FK_OK   # disarmed again
