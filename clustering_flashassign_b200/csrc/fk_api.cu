@@ -1,6 +1,7 @@
 // The extern "C" surface of libfk (declared in include/fk.h): argument checks,
 // dispatch to the kernels, the Lloyd loop and its streamed (out-of-core) path.
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "fk_internal.h"
@@ -32,6 +33,18 @@ int check_shape(int B, long long N, int K, int d, int dtype) {
   if (dtype != FK_F32 && (d * 2) % 16 != 0)
     return set_error(FK_EINVAL, "fp16/bf16 rows must be a multiple of 16 bytes (d % 8 == 0)");
   return FK_OK;
+}
+
+// Options with the environment's defaults: FK_VERBOSE=1 turns the per-iteration
+// line on, FK_CHUNK_POINTS sets the streamed chunk size when the caller left it 0.
+fk_options options_of(const fk_options *opts) {
+  fk_options o{FK_HOST_AUTO, 0, 0};
+  if (opts) o = *opts;
+  if (const char *e = getenv("FK_VERBOSE"))
+    if (atoi(e) != 0) o.verbose = 1;
+  if (o.chunk_points <= 0)
+    if (const char *e = getenv("FK_CHUNK_POINTS")) o.chunk_points = atoll(e);
+  return o;
 }
 
 int check_ptr(const void *p, const char *name, bool aligned16) {
@@ -386,7 +399,7 @@ int fk_lloyd_step_partial(const fk_shape *shape, const void *x, const float *xn,
   FK_TRY(check_ptr(ids, "ids", false));
   FK_TRY(check_ptr(sums, "sums", false));
   FK_TRY(check_ptr(counts, "counts", false));
-  const fk_options o = opts ? *opts : fk_options{FK_HOST_AUTO, 0, 0};
+  const fk_options o = options_of(opts);
   Workspace *ws;
   FK_TRY(workspace_for(s, &ws));
   const long long Kpad = kpad_of(K);
@@ -450,8 +463,7 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
   FK_TRY(check_ptr(ids, "ids", false));
   FK_TRY(check_ptr(centers, "centers", true));
   if (max_iter < 0) return set_error(FK_EINVAL, "max_iter must be >= 0");
-  fk_options o{FK_HOST_AUTO, 0, 0};
-  if (opts) o = *opts;
+  const fk_options o = options_of(opts);
   const int B = sh.B, K = sh.K, d = sh.d, dtype = sh.dtype;
   const long long N = sh.N;
   const size_t es = esize(dtype);

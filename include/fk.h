@@ -79,8 +79,10 @@ typedef enum {
 
 typedef struct {
   int host_mode;          /* fk_host_mode; used only when x is host memory */
-  long long chunk_points; /* streamed path: points per chunk; 0 = 2^24 */
-  int verbose;            /* 1: one line per iteration on stderr */
+  long long chunk_points; /* streamed path: points per chunk; 0 = FK_CHUNK_POINTS
+                             from the environment, else 2^24 */
+  int verbose;            /* 1: one line per iteration on stderr (also with
+                             FK_VERBOSE=1 in the environment) */
 } fk_options;
 
 /*
