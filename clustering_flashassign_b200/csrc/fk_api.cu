@@ -133,8 +133,14 @@ int assign_f32_tc(Workspace *ws, const float *x, const float *c, const float *x3
   // tile's chunks: one work item per (tile, chunk), consecutive CTAs sharing a
   // tile's reads, merged through per-point keys
   FK_TRY(ensure_zeroed(ws->keys64, (size_t)B * N * sizeof(unsigned long long), s));
-  return launch_assign_tc(x3, ws->c3.p, ws->cn.p, nullptr, FK_F32, B, N, K, d3, Kpad, ids, ws->err, s,
-                          hist, (unsigned long long *)ws->keys64.p);
+  // the keys are cleared by the kernel that turns them into ids; if an earlier
+  // call stopped between the two launches they are cleared here
+  if (ws->keys_dirty) FK_CUDA(cudaMemsetAsync(ws->keys64.p, 0, ws->keys64.bytes, s));
+  ws->keys_dirty = true;
+  FK_TRY(launch_assign_tc(x3, ws->c3.p, ws->cn.p, nullptr, FK_F32, B, N, K, d3, Kpad, ids, ws->err, s,
+                          hist, (unsigned long long *)ws->keys64.p));
+  ws->keys_dirty = false;
+  return FK_OK;
 }
 
 int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const void *cnx,

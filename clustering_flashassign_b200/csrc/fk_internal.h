@@ -56,6 +56,7 @@ struct Workspace {
   DevBuf xres, init_dev, ids_dev, centers_dev, chunk[2], gsum, gcounts, xn, ids_alt;
   DevBuf x3, c3;                  // 3xTF32 operands of the fp32 tensor-core assign
   DevBuf keys64;                  // split-d per-point argmax keys, kept zeroed
+  bool keys_dirty = false;        // an assign wrote keys64 that nothing has cleared yet
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
   cudaEvent_t shift_ev = nullptr;  // the max-shift copy of the Lloyd loop has landed

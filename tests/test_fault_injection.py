@@ -119,3 +119,27 @@ def test_fault_from_the_environment():
     out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr
     assert "status 2" in out.stdout and "recovered" in out.stdout   # FK_ENOMEM == 2
+
+
+def test_fp32_tensor_core_assign_recovers_after_a_stop_between_its_launches():
+    """The fp32 tensor-core assign merges chunks through per-point keys that the
+    next kernel turns into ids and clears.  A call stopped right after the assign
+    kernel (its fourth launch: two row splits, the norm rows, the assign) leaves
+    keys behind; the next call must clear them and give the right ids."""
+    import clustering_flashassign_b200 as fk
+    B, N, K, d = 1, 2000, 600, 64            # K * d >= 16384: tensor cores, 3 chunks
+    x, _, c = case(B, N, K, d, "f32", mean_std=4.0, seed=83)
+    xd, cd = to_dev(x, "f32"), to_dev(c, "f32")
+    ids = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    fk.fk_inject_fault(fk.FK_FAULT_LAUNCH, 4)
+    with pytest.raises(fk.FkError):
+        fk.fk_assign(xd, cd, ids)
+    torch.cuda.synchronize()
+    # other centroids: a stale key of the stopped call (a value under the old
+    # centroids) would win the merge and leave a wrong id
+    c2 = (c[:, ::-1] * 0.5 + 1.0).astype(np.float32)
+    ids.fill_(-1)
+    fk.fk_assign(xd, to_dev(np.ascontiguousarray(c2), "f32"), ids)
+    torch.cuda.synchronize()
+    assert fk.fk_device_error() == 0
+    check_ids(ids.cpu().numpy(), x, "f32", c2.astype(np.float64))
