@@ -22,7 +22,7 @@ pytestmark = pytest.mark.gpu
 TORCH_DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 
 
-@pytest.mark.parametrize("name", ["tiny", "api", "zipf", "splitd"])
+@pytest.mark.parametrize("name", ["tiny", "api", "zipf", "splitd", "f32large"])
 def test_full_size_workload(name):
     import clustering_flashassign_b200 as fk
     w = synthdata.WORKLOADS[name]
