@@ -230,7 +230,8 @@ __global__ void __launch_bounds__(kSortThreads) k_scan_tiles(uint32_t *__restric
 // It writes vals_out[pos] = vals_in ? vals_in[i] : i and keys_out[pos] = key
 // (each when not NULL), or the pair kv_out[pos] = (key, value): one 8-byte
 // store per point where the update needs both.  The CTA of tile 0 also writes
-// offsets_out[b] (when not NULL).  zero_g: the tile's row of G is zeroed once
+// offsets_out[b] (when not NULL) and -1 entries past the counted points (when
+// an id was out of range).  zero_g: the tile's row of G is zeroed once
 // read, so a histogram that the assign accumulates starts from zero again.
 __global__ void __launch_bounds__(kSortThreads) k_tile_scatter(
     const int32_t *__restrict__ keys, const int32_t *__restrict__ vals_in, int N, int K, int T,
@@ -282,6 +283,17 @@ __global__ void __launch_bounds__(kSortThreads) k_tile_scatter(
   int32_t *ko = keys_out ? keys_out + (size_t)b * N : nullptr;
   int32_t *vo = vals_out ? vals_out + (size_t)b * N : nullptr;
   int2 *kvo = kv_out ? kv_out + (size_t)b * N : nullptr;
+  if (tile == 0) {
+    // ids outside [0, K) are counted nowhere, so the counted points end before
+    // N; the positions past them get -1 (key, value) instead of whatever an
+    // earlier call left there.  Nothing to do when every id is valid.
+    const int total = (int)(tb[bins - 1] + (uint32_t)counts[(size_t)b * bins + bins - 1]);
+    for (int i = total + threadIdx.x; i < N; i += kSortThreads) {
+      if (kvo) kvo[i] = make_int2(-1, -1);
+      if (vo) vo[i] = -1;
+      if (ko) ko[i] = -1;
+    }
+  }
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
   for (int r = 0; r < kRounds; ++r) {
@@ -368,14 +380,11 @@ int bits_for(int K) {
 }
 
 int set_attrs() {
-  static bool done = false;
-  if (done) return FK_OK;
   const int hist_max = kSortWarps * (1 << kMaxDigitBits) * 4;
   const int scat_max = (kSortWarps + 1) * (1 << kMaxDigitBits) * 4;
-  FK_CUDA(cudaFuncSetAttribute(k_tile_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, hist_max));
-  FK_CUDA(cudaFuncSetAttribute(k_tile_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, scat_max));
-  FK_CUDA(cudaFuncSetAttribute(k_count, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
-  done = true;
+  FK_TRY(set_smem_limit((const void *)k_tile_hist, hist_max));
+  FK_TRY(set_smem_limit((const void *)k_tile_scatter, scat_max));
+  FK_TRY(set_smem_limit((const void *)k_count, 64 * 1024));
   return FK_OK;
 }
 
@@ -461,7 +470,9 @@ int run_sort(Workspace *ws, const int32_t *ids, int B, long long N_, int K, int3
   int32_t *dcnt = (int32_t *)ws->digit_off.p;
   PassCfg p1{0, (1u << lo) - 1u, 1 << lo, lo, true};
   FK_TRY(one_pass(ws, ids, nullptr, B, N, K, T, p1, dcnt, nullptr, kt, vt, nullptr, s));
-  PassCfg p2{lo, (1u << hi) - 1u, 1 << hi, hi, false};
+  // the second pass validates its keys too, so the -1 entries that stand for
+  // out-of-range ids past the first pass's counted points are dropped again
+  PassCfg p2{lo, (1u << hi) - 1u, 1 << hi, hi, true};
   FK_TRY(one_pass(ws, kt, vt, B, N, K, T, p2, dcnt, nullptr, nullptr, perm, kv_out, s));
   // cluster counts and offsets (a pass's digit totals are not cluster totals)
   FK_CUDA(cudaMemsetAsync(cnt, 0, (size_t)B * K * sizeof(int32_t), s));

@@ -141,6 +141,9 @@ int fk_update(const void *x, const int32_t *ids, int B, long long N, int K, int 
  * (sort the assignment vector by cluster id into contiguous segments).
  *   ids (B, N) int32 in [0, K), device.  counts, offsets (B, K) int32 out,
  *   device, each may be NULL.  perm (B, N) int32 out, device.
+ * ids outside [0, K) are a caller error: they are counted nowhere, the
+ * entries of perm past a batch's counted points are -1, and the device error
+ * word records FK_EINVAL.
  */
 int fk_sort(const int32_t *ids, int B, long long N, int K, int32_t *counts, int32_t *offsets,
             int32_t *perm, fk_stream_t stream);

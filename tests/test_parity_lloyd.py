@@ -135,17 +135,44 @@ def test_host_buffers_resident_and_streamed():
         check_centers(cen.numpy(), r["centers"], "f16")
 
 
-def test_out_of_range_ids_are_reported_not_faulted():
+@pytest.mark.parametrize("K", [20, 5000])   # one counting pass; two passes (K > 4096)
+def test_out_of_range_ids_are_counted_nowhere(K):
+    """Two ids outside [0, K), after a valid call has left full sort buffers
+    behind: the error is reported, not faulted, and every other point's result
+    is the oracle's over the valid points alone -- counts, centroids and the
+    stable permutation -- with -1 in perm past the counted points."""
     import clustering_flashassign_b200 as fk
-    B, N, K, d = 1, 500, 20, 16
-    x, idx, c0 = case(B, N, K, d, "f16")
-    ids = torch.randint(0, K, (B, N), dtype=torch.int32, device="cuda")
-    ids[0, 7] = K
-    ids[0, 9] = -1
-    cen = torch.from_numpy(synthdata.to_f64(c0, "f16").astype(np.float32)).cuda()
-    fk.fk_update(to_dev(x, "f16"), ids, cen)
+    B, N, d = 1, 12000, 16
+    x, _, c0 = case(B, N, K, d, "f16", seed=53)
+    xd = to_dev(x, "f16")
+    c64 = synthdata.to_f64(c0, "f16")
+    rng = np.random.default_rng(53)
+    ok = torch.from_numpy(rng.integers(0, K, (B, N)).astype(np.int32)).cuda()
+    fk.fk_update(xd, ok, torch.from_numpy(c64.astype(np.float32)).cuda())
+    fk.fk_sort(ok, K, torch.empty((B, N), dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    assert fk.fk_device_error() == fk.FK_OK
+    g = rng.integers(0, K, (B, N)).astype(np.int32)
+    g[0, 7] = K
+    g[0, 9] = -1
+    ids = torch.from_numpy(g).cuda()
+    cen = torch.from_numpy(c64.astype(np.float32)).cuda()
+    counts = torch.empty((B, K), dtype=torch.int32, device="cuda")
+    fk.fk_update(xd, ids, cen, counts)
+    perm = torch.full((B, N), 12345, dtype=torch.int32, device="cuda")
+    fk.fk_sort(ids, K, perm)
+    torch.cuda.synchronize()
     assert fk.fk_device_error() == fk.FK_EINVAL
     assert fk.fk_device_error() == fk.FK_OK  # reading clears it
+    keep = (g[0] >= 0) & (g[0] < K)
+    new, rc, _, _ = oracle.update(x[:, keep], "f16", g[:, keep], c64)
+    np.testing.assert_array_equal(counts.cpu().numpy(), rc)
+    check_centers(cen.cpu().numpy(), new, "f16")
+    _, operm = oracle.sort(g[:, keep], K)
+    nv = int(keep.sum())
+    p = perm.cpu().numpy()[0]
+    np.testing.assert_array_equal(p[:nv], np.flatnonzero(keep)[operm[0]])
+    assert (p[nv:] == -1).all()
 
 
 def test_repeated_runs_are_bit_identical():
