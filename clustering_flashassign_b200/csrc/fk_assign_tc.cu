@@ -759,12 +759,7 @@ template <typename T, bool RESIDENT, int KB, int STAGES>
 int launch_variant(const CUtensorMap &tmx, const CUtensorMap &tmc, const CUtensorMap &tme,
                    const TcArgs &a, int grid, cudaStream_t s) {
   using L = Layout<RESIDENT, KB, STAGES>;
-  static bool attr = false;
-  if (!attr) {
-    FK_CUDA(cudaFuncSetAttribute(k_flash_assign<T, RESIDENT, KB, STAGES>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc));
-    attr = true;
-  }
+  FK_TRY(set_smem_limit((const void *)k_flash_assign<T, RESIDENT, KB, STAGES>, (int)L::kAlloc));
   FK_CUDA(launch_pdl(k_flash_assign<T, RESIDENT, KB, STAGES>, dim3(grid), dim3(kThreads), L::kAlloc, s, tmx, tmc,
                      tme, a));
   FK_TRY(launched());

@@ -80,6 +80,9 @@ int cuda_status(cudaError_t e, const char *what);
 int ensure(DevBuf &b, size_t bytes);               // grow-only device buffer
 int ensure_zeroed(DevBuf &b, size_t bytes, cudaStream_t s);  // zero-filled when (re)allocated
 int workspace_for(cudaStream_t s, Workspace **out);
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per (device, kernel).
+int set_smem_limit(const void *func, int bytes);
 
 // Launch accounting and event timing.
 // Launch accounting; returns FK_ECUDA when an injected launch fault fires.

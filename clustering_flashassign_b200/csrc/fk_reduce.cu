@@ -311,12 +311,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_segreduce16(const T *__restrict
 template <typename T>
 int launch16(const void *x, const int2 *kv, int B, int N, int K, int d, float *sums, float *first,
              cudaStream_t s) {
-  static bool attr = false;
   const int shm = kWarps * 2 * kBufBytes;
-  if (!attr) {
-    FK_CUDA(cudaFuncSetAttribute(k_segreduce16<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, shm));
-    attr = true;
-  }
+  FK_TRY(set_smem_limit((const void *)k_segreduce16<T>, shm));
   const int pieces = (N + kPiece - 1) / kPiece;
   const int colblocks = (d + 127) / 128;
   const long long items = (long long)B * pieces * colblocks;

@@ -4,6 +4,7 @@
 #include <cstdlib>
 #include <map>
 #include <mutex>
+#include <set>
 #include <utility>
 #include <vector>
 
@@ -70,6 +71,19 @@ int ensure(DevBuf &b, size_t bytes) {
     want = bytes;
   }
   b.bytes = want;
+  return FK_OK;
+}
+
+int set_smem_limit(const void *func, int bytes) {
+  // the attribute belongs to the kernel as loaded on the current device
+  static std::mutex mu;
+  static std::set<std::pair<int, const void *>> done;
+  int dev = 0;
+  FK_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count({dev, func})) return FK_OK;
+  FK_CUDA(cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  done.insert({dev, func});
   return FK_OK;
 }
 
