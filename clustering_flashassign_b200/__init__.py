@@ -21,6 +21,7 @@ the loop that joins them with an all-reduce is clustering_flashassign_b200.dist)
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -117,6 +118,15 @@ def _stream(stream):
     return ctypes.c_void_p(int(stream))
 
 
+def _on(*tensors):
+    """Make the device of the first CUDA tensor current for the call (the library
+    works on the current device, and the default stream is that device's)."""
+    for t in tensors:
+        if t is not None and t.is_cuda:
+            return torch.cuda.device(t.device)
+    return contextlib.nullcontext()
+
+
 def _ptr(t):
     if t is None:
         return None
@@ -135,8 +145,9 @@ def fk_assign(x: torch.Tensor, c: torch.Tensor, ids: torch.Tensor, stream=None) 
     """ids[b,i] = argmin_k ||c_k||^2 - 2 x_i.c_k (lowest k on ties)."""
     B, N, d = x.shape
     K = c.shape[1]
-    _check(lib.fk_assign(_ptr(x), _ptr(c), B, N, K, d, _dtype_code(x), _ptr(ids), _stream(stream)),
-           "fk_assign")
+    with _on(x, c, ids):
+        _check(lib.fk_assign(_ptr(x), _ptr(c), B, N, K, d, _dtype_code(x), _ptr(ids), _stream(stream)),
+               "fk_assign")
     return ids
 
 
@@ -144,8 +155,9 @@ def fk_assign_noalloc(x: torch.Tensor, c: torch.Tensor, ids: torch.Tensor, strea
     """fk_assign that allocates no device memory (static scratch; see include/fk.h)."""
     B, N, d = x.shape
     K = c.shape[1]
-    _check(lib.fk_assign_noalloc(_ptr(x), _ptr(c), B, N, K, d, _dtype_code(x), _ptr(ids),
-                                 _stream(stream)), "fk_assign_noalloc")
+    with _on(x, c, ids):
+        _check(lib.fk_assign_noalloc(_ptr(x), _ptr(c), B, N, K, d, _dtype_code(x), _ptr(ids),
+                                     _stream(stream)), "fk_assign_noalloc")
     return ids
 
 
@@ -154,8 +166,9 @@ def fk_update(x: torch.Tensor, ids: torch.Tensor, centers: torch.Tensor, counts=
     """Sort-inverse update: centers (B,K,d) fp32 in/out, counts (B,K) int32 out."""
     B, N, d = x.shape
     K = centers.shape[1]
-    _check(lib.fk_update(_ptr(x), _ptr(ids), B, N, K, d, _ptr(centers), _ptr(counts),
-                         _stream(stream), _dtype_code(x), _ptr(max_shift)), "fk_update")
+    with _on(x, ids, centers):
+        _check(lib.fk_update(_ptr(x), _ptr(ids), B, N, K, d, _ptr(centers), _ptr(counts),
+                             _stream(stream), _dtype_code(x), _ptr(max_shift)), "fk_update")
     return centers
 
 
@@ -163,8 +176,9 @@ def fk_sort(ids: torch.Tensor, K: int, perm: torch.Tensor, counts=None, offsets=
             stream=None) -> torch.Tensor:
     """Stable counting sort of ids: perm lists point indices ordered by (id, index)."""
     B, N = ids.shape
-    _check(lib.fk_sort(_ptr(ids), B, N, K, _ptr(counts), _ptr(offsets), _ptr(perm), _stream(stream)),
-           "fk_sort")
+    with _on(ids, perm):
+        _check(lib.fk_sort(_ptr(ids), B, N, K, _ptr(counts), _ptr(offsets), _ptr(perm), _stream(stream)),
+               "fk_sort")
     return perm
 
 
@@ -177,25 +191,28 @@ def fk_lloyd(x: torch.Tensor, init_centers: torch.Tensor, max_iter: int, tol: fl
     shape = FkShape(B, N, K, d, _dtype_code(x))
     opts = FkOptions(host_mode, chunk_points, 1 if verbose else 0)
     iters = ctypes.c_int(0)
-    _check(lib.fk_lloyd(ctypes.byref(shape), _ptr(x), _ptr(init_centers), int(max_iter), float(tol),
-                        _ptr(ids), _ptr(centers), _stream(stream), ctypes.byref(iters),
-                        ctypes.byref(opts)), "fk_lloyd")
+    with _on(x, init_centers, ids, centers):
+        _check(lib.fk_lloyd(ctypes.byref(shape), _ptr(x), _ptr(init_centers), int(max_iter), float(tol),
+                            _ptr(ids), _ptr(centers), _stream(stream), ctypes.byref(iters),
+                            ctypes.byref(opts)), "fk_lloyd")
     return iters.value
 
 
 def fk_point_norms(x: torch.Tensor, xn: torch.Tensor, stream=None) -> torch.Tensor:
     """xn (B, N) fp32 = ||x[b, i]||^2 of fp16 / bf16 points (B, N, d)."""
     B, N, d = x.shape
-    _check(lib.fk_point_norms(_ptr(x), B, N, d, _dtype_code(x), _ptr(xn), _stream(stream)),
-           "fk_point_norms")
+    with _on(x, xn):
+        _check(lib.fk_point_norms(_ptr(x), B, N, d, _dtype_code(x), _ptr(xn), _stream(stream)),
+               "fk_point_norms")
     return xn
 
 
 def fk_init_centers(init: torch.Tensor, centers: torch.Tensor, stream=None) -> torch.Tensor:
     """centers (B, K, d) fp32 = init (B, K, d) in the points' dtype, widened exactly."""
     B, K, d = init.shape
-    _check(lib.fk_init_centers(_ptr(init), B, K, d, _dtype_code(init), _ptr(centers), _stream(stream)),
-           "fk_init_centers")
+    with _on(init, centers):
+        _check(lib.fk_init_centers(_ptr(init), B, K, d, _dtype_code(init), _ptr(centers), _stream(stream)),
+               "fk_init_centers")
     return centers
 
 
@@ -208,9 +225,10 @@ def fk_lloyd_step_partial(x: torch.Tensor, xn, centers_dt: torch.Tensor, ids: to
     K = centers_dt.shape[1]
     shape = FkShape(B, N, K, d, _dtype_code(x))
     opts = FkOptions(FK_HOST_AUTO, chunk_points, 0)
-    _check(lib.fk_lloyd_step_partial(ctypes.byref(shape), _ptr(x), _ptr(xn), _ptr(centers_dt), _ptr(ids),
-                                     _ptr(sums), _ptr(counts), _stream(stream), ctypes.byref(opts)),
-           "fk_lloyd_step_partial")
+    with _on(x, centers_dt, ids, sums):
+        _check(lib.fk_lloyd_step_partial(ctypes.byref(shape), _ptr(x), _ptr(xn), _ptr(centers_dt), _ptr(ids),
+                                         _ptr(sums), _ptr(counts), _stream(stream), ctypes.byref(opts)),
+               "fk_lloyd_step_partial")
 
 
 def fk_update_finalize(sums: torch.Tensor, counts: torch.Tensor, centers: torch.Tensor,
@@ -218,8 +236,9 @@ def fk_update_finalize(sums: torch.Tensor, counts: torch.Tensor, centers: torch.
     """centers = sums / counts where counts > 0 (else unchanged); centers_dt = rounded copy."""
     B, K, d = centers.shape
     code = _dtype_code(centers_dt) if centers_dt is not None else DTYPES[dtype or torch.float32]
-    _check(lib.fk_update_finalize(_ptr(sums), _ptr(counts), B, K, d, code, _ptr(centers), _ptr(centers_dt),
-                                  _ptr(max_shift), _stream(stream)), "fk_update_finalize")
+    with _on(sums, counts, centers):
+        _check(lib.fk_update_finalize(_ptr(sums), _ptr(counts), B, K, d, code, _ptr(centers), _ptr(centers_dt),
+                                      _ptr(max_shift), _stream(stream)), "fk_update_finalize")
     return centers
 
 

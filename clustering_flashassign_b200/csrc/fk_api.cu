@@ -54,6 +54,32 @@ int check_ptr(const void *p, const char *name, bool aligned16) {
   return FK_OK;
 }
 
+// A pointer that the current device's kernels read or write: memory of this
+// device, or managed memory.  Host memory and another device's memory are
+// refused here instead of reaching a kernel.
+int check_dev(const void *p, const char *name) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return set_error(FK_EINVAL, std::string(name) + " must be device memory");
+  }
+  if (at.type == cudaMemoryTypeManaged) return FK_OK;
+  if (at.type != cudaMemoryTypeDevice) return set_error(FK_EINVAL, std::string(name) + " must be device memory");
+  int dev = 0;
+  FK_CUDA(cudaGetDevice(&dev));
+  if (at.device != dev)
+    return set_error(FK_EINVAL, std::string(name) + " is memory of device " + std::to_string(at.device) +
+                                    ", not of the current device " + std::to_string(dev));
+  return FK_OK;
+}
+
+int check_dev_opt(const void *p, const char *name) { return p ? check_dev(p, name) : FK_OK; }
+
+// An argument that may be host or device memory: device memory must be this device's.
+int check_if_dev(const void *p, Loc where, const char *name) {
+  return where == LOC_DEVICE ? check_dev(p, name) : FK_OK;
+}
+
 int read_device_error(Workspace *ws, cudaStream_t s) {
   int h = 0;
   FK_CUDA(cudaMemcpyAsync(&h, ws->err, sizeof(int), cudaMemcpyDeviceToHost, s));
@@ -330,6 +356,9 @@ int fk_assign(const void *x, const void *c, int B, long long N, int K, int d, in
   FK_TRY(check_ptr(x, "x", tc));
   FK_TRY(check_ptr(c, "c", tc));
   FK_TRY(check_ptr(ids, "ids", false));
+  FK_TRY(check_dev(x, "x"));
+  FK_TRY(check_dev(c, "c"));
+  FK_TRY(check_dev(ids, "ids"));
   Workspace *ws;
   FK_TRY(workspace_for(s, &ws));
   const long long Kpad = kpad_of(K);
@@ -349,6 +378,11 @@ int fk_update(const void *x, const int32_t *ids, int B, long long N, int K, int 
   FK_TRY(check_ptr(x, "x", true));
   FK_TRY(check_ptr(ids, "ids", false));
   FK_TRY(check_ptr(centers, "centers", true));
+  FK_TRY(check_dev(x, "x"));
+  FK_TRY(check_dev(ids, "ids"));
+  FK_TRY(check_dev(centers, "centers"));
+  FK_TRY(check_dev_opt(counts, "counts"));
+  FK_TRY(check_dev_opt(max_shift, "max_shift"));
   Workspace *ws;
   FK_TRY(workspace_for(s, &ws));
   FK_TRY(do_update(ws, x, ids, B, N, K, d, dtype, centers, counts, nullptr, nullptr, kpad_of(K), s));
@@ -363,6 +397,10 @@ int fk_sort(const int32_t *ids, int B, long long N, int K, int32_t *counts, int3
   FK_TRY(check_shape(B, N, K, 8, FK_F32));
   FK_TRY(check_ptr(ids, "ids", false));
   FK_TRY(check_ptr(perm, "perm", false));
+  FK_TRY(check_dev(ids, "ids"));
+  FK_TRY(check_dev(perm, "perm"));
+  FK_TRY(check_dev_opt(counts, "counts"));
+  FK_TRY(check_dev_opt(offsets, "offsets"));
   Workspace *ws;
   FK_TRY(workspace_for(s, &ws));
   PhaseTimer t(PH_SORT, s);
@@ -376,6 +414,8 @@ int fk_point_norms(const void *x, int B, long long N, int d, int dtype, float *x
   if (dtype == FK_F32) return set_error(FK_EUNSUPPORTED, "point norms serve the fp16 / bf16 assign");
   FK_TRY(check_ptr(x, "x", true));
   FK_TRY(check_ptr(xn, "xn", false));
+  FK_TRY(check_dev(x, "x"));
+  FK_TRY(check_dev(xn, "xn"));
   return launch_point_norms(x, dtype, (long long)B * N, d, xn, s);
 }
 
@@ -385,6 +425,8 @@ int fk_init_centers(const void *init, int B, int K, int d, int dtype, float *cen
   FK_TRY(check_shape(B, K, K, d, dtype));
   FK_TRY(check_ptr(init, "init", false));
   FK_TRY(check_ptr(centers, "centers", false));
+  FK_TRY(check_dev(init, "init"));
+  FK_TRY(check_dev(centers, "centers"));
   Workspace *ws;
   FK_TRY(workspace_for(s, &ws));
   return launch_init_centers(init, dtype, B, K, d, kpad_of(K), centers, nullptr, nullptr, ws->err, s);
@@ -405,6 +447,11 @@ int fk_lloyd_step_partial(const fk_shape *shape, const void *x, const float *xn,
   FK_TRY(check_ptr(ids, "ids", false));
   FK_TRY(check_ptr(sums, "sums", false));
   FK_TRY(check_ptr(counts, "counts", false));
+  FK_TRY(check_dev(centers_dt, "centers_dt"));
+  FK_TRY(check_dev(ids, "ids"));
+  FK_TRY(check_dev(sums, "sums"));
+  FK_TRY(check_dev(counts, "counts"));
+  FK_TRY(check_dev_opt(xn, "xn"));
   const fk_options o = options_of(opts);
   Workspace *ws;
   FK_TRY(workspace_for(s, &ws));
@@ -417,6 +464,7 @@ int fk_lloyd_step_partial(const fk_shape *shape, const void *x, const float *xn,
   }
   const Loc lx = locate(x);
   if (lx == LOC_HOST_PAGEABLE) return set_error(FK_EINVAL, "x must be device or pinned host memory");
+  FK_TRY(check_if_dev(x, lx, "x"));
   if (lx == LOC_HOST_PINNED) {
     long long chunk = o.chunk_points > 0 ? o.chunk_points : (1LL << 24);
     if (chunk > N) chunk = N;
@@ -444,6 +492,11 @@ int fk_update_finalize(const float *sums, const int32_t *counts, int B, int K, i
   FK_TRY(check_ptr(sums, "sums", false));
   FK_TRY(check_ptr(counts, "counts", false));
   FK_TRY(check_ptr(centers, "centers", true));
+  FK_TRY(check_dev(sums, "sums"));
+  FK_TRY(check_dev(counts, "counts"));
+  FK_TRY(check_dev(centers, "centers"));
+  if (dtype != FK_F32) FK_TRY(check_dev_opt(centers_dt, "centers_dt"));
+  FK_TRY(check_dev_opt(max_shift, "max_shift"));
   Workspace *ws;
   FK_TRY(workspace_for(s, &ws));
   FK_CUDA(cudaMemsetAsync(ws->maxshift, 0, sizeof(unsigned), s));
@@ -480,6 +533,10 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
   FK_TRY(workspace_for(s, &ws));
 
   const Loc lx = locate(x), li = locate(init_centers), lids = locate(ids), lc = locate(centers);
+  FK_TRY(check_if_dev(x, lx, "x"));
+  FK_TRY(check_if_dev(init_centers, li, "init_centers"));
+  FK_TRY(check_if_dev(ids, lids, "ids"));
+  FK_TRY(check_if_dev(centers, lc, "centers"));
   const void *init_dev = init_centers;
   if (li != LOC_DEVICE) {
     FK_TRY(ensure(ws->init_dev, cbytes));

@@ -31,7 +31,10 @@
  *   - Every call returns an fk_status.  Nothing throws across the ABI.
  *     FK_EINVAL: a size <= 0, K > N, N or K beyond 2^31-1, a null pointer,
  *     an unknown dtype, or (fp16 / bf16) d*2 not a multiple of 16 bytes or a
- *     pointer not 16-byte aligned.  FK_EUNSUPPORTED: a shape beyond the
+ *     pointer not 16-byte aligned; also a pointer documented as device memory
+ *     that is host memory or memory of another device than the current one
+ *     (device memory passed where host memory is allowed must be the current
+ *     device's too; managed memory is accepted).  FK_EUNSUPPORTED: a shape beyond the
  *     limits stated per call.  FK_ECUDA: a CUDA runtime error (see
  *     fk_last_error()).  FK_ETIMEOUT: a kernel's bounded wait expired (the
  *     kernel recorded it in the device error word and returned; see
@@ -262,6 +265,9 @@ int fk_update_finalize(const float *sums, const int32_t *counts, int B, int K, i
  *   Limit: B * Kpad <= 131072 for fp16 / bf16, Kpad = K rounded up to a
  *   multiple of 256; larger shapes return FK_EUNSUPPORTED.  fp32 needs no
  *   scratch and has no such limit.
+ *   Unlike the other calls, this one does not check that x, c and ids are
+ *   memory of the current device (it makes no runtime query that a stream
+ *   capture might refuse): the caller guarantees it.
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
  *   before any stream capture.

@@ -129,3 +129,31 @@ def test_bounded_wait_expires_and_the_context_survives():
     g, err = _assign(x, c, "f16")
     assert err == 0
     check_ids(g, x, "f16", synthdata.to_f64(c, "f16"))
+
+
+def test_host_memory_where_device_memory_is_required_is_refused():
+    """Host buffers (pageable or pinned) passed where the ABI wants device
+    memory return FK_EINVAL from the host-side check, before any launch; the
+    device error word stays clean and the next valid call runs."""
+    import clustering_flashassign_b200 as fk
+    L = fk.lib
+    B, N, K, d = 1, 512, 16, 64
+    x, _, c = case(B, N, K, d, "f16", seed=61)
+    xd, cd = to_dev(x, "f16"), to_dev(c, "f16")
+    ids = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    for xh in (torch.from_numpy(x).clone(), torch.from_numpy(x).pin_memory()):
+        st = L.fk_assign(xh.data_ptr(), cd.data_ptr(), B, N, K, d, fk.FK_F16, ids.data_ptr(), s)
+        assert st == fk.FK_EINVAL and "x must be device memory" in fk.fk_last_error()
+    ids_h = torch.zeros((B, N), dtype=torch.int32)
+    cen = torch.zeros((B, K, d), dtype=torch.float32, device="cuda")
+    st = L.fk_update(xd.data_ptr(), ids_h.data_ptr(), B, N, K, d, cen.data_ptr(), None, s, fk.FK_F16, None)
+    assert st == fk.FK_EINVAL and "ids must be device memory" in fk.fk_last_error()
+    perm_h = torch.empty((B, N), dtype=torch.int32)
+    st = L.fk_sort(ids.data_ptr(), B, N, K, None, None, perm_h.data_ptr(), s)
+    assert st == fk.FK_EINVAL and "perm must be device memory" in fk.fk_last_error()
+    torch.cuda.synchronize()
+    assert fk.fk_device_error() == 0
+    got, err = _assign(x, c, "f16")
+    assert err == 0
+    check_ids(got, x, "f16", synthdata.to_f64(c, "f16"))
