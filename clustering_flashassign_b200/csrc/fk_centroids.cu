@@ -133,11 +133,12 @@ __device__ __forceinline__ float seg_sum(const float *sums, const float *first, 
 }
 
 // One warp per centroid (no grid-stride loop, so every centroid's loads are
-// in flight at once).  With d % 4 == 0 lane l handles elements 4l..4l+3,
+// in flight at once); held to 32 registers so that eight CTAs (64 warps)
+// share an SM: the kernel waits on loads, and more warps hide more of them.  With d % 4 == 0 lane l handles elements 4l..4l+3,
 // 4l+128.. with 16-byte loads and stores; the arithmetic order per element is
 // the same as in the scalar form.
 template <typename T, bool V4, bool FROM_PIECES>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 8)
     k_finalize(const float *__restrict__ sums, const float *__restrict__ first, int pieces,
                const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets,
                float *__restrict__ centers, T *__restrict__ ch, T *__restrict__ cnx, int B, int K,
