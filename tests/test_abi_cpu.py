@@ -121,3 +121,34 @@ def test_fault_injection_arguments():
     assert L.fk_inject_fault(fk.FK_FAULT_ALLOC, 0) == fk.FK_EINVAL
     assert L.fk_inject_fault(fk.FK_FAULT_ALLOC, 3) == fk.FK_OK
     assert L.fk_inject_fault(fk.FK_FAULT_NONE, 1) == fk.FK_OK   # disarmed again
+
+
+def test_binding_runs_each_call_on_its_first_cuda_tensors_device(monkeypatch):
+    """The wrappers enter torch.cuda.device(...) of the first CUDA tensor among
+    their arguments (the library works on the current device); host-only
+    arguments switch nothing."""
+    import clustering_flashassign_b200 as fk
+    seen = []
+
+    class Recorder:
+        def __init__(self, dev):
+            seen.append(dev)
+
+        def __enter__(self):
+            return self
+
+        def __exit__(self, *exc):
+            return False
+
+    class Tensor:  # stands in for a torch tensor on `dev` (None: host memory)
+        def __init__(self, dev):
+            self.is_cuda = dev is not None
+            self.device = dev
+
+    monkeypatch.setattr(fk.torch.cuda, "device", Recorder)
+    with fk._on(Tensor(None), None, Tensor("cuda:1"), Tensor("cuda:0")):
+        pass
+    assert seen == ["cuda:1"]
+    with fk._on(Tensor(None), None):
+        pass
+    assert seen == ["cuda:1"]
