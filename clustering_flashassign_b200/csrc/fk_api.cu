@@ -440,17 +440,27 @@ int fk_lloyd_step_partial(const fk_shape *shape, const void *x, const float *xn,
   const fk_shape sh = *shape;
   const int B = sh.B, K = sh.K, d = sh.d, dtype = sh.dtype;
   const long long N = sh.N;
-  FK_TRY(check_shape(B, N, K, d, dtype));
+  // a rank's block of a larger problem may hold fewer points than there are
+  // clusters, or none: only the whole problem needs K <= N
+  if (N < 0) return set_error(FK_EINVAL, "N must be >= 0");
+  FK_TRY(check_shape(B, N > K ? N : K, K, d, dtype));
   const bool tc = dtype != FK_F32;
-  FK_TRY(check_ptr(x, "x", tc));
+  if (N > 0) {
+    FK_TRY(check_ptr(x, "x", tc));
+    FK_TRY(check_ptr(ids, "ids", false));
+  }
   FK_TRY(check_ptr(centers_dt, "centers_dt", tc));
-  FK_TRY(check_ptr(ids, "ids", false));
   FK_TRY(check_ptr(sums, "sums", false));
   FK_TRY(check_ptr(counts, "counts", false));
   FK_TRY(check_dev(centers_dt, "centers_dt"));
-  FK_TRY(check_dev(ids, "ids"));
   FK_TRY(check_dev(sums, "sums"));
   FK_TRY(check_dev(counts, "counts"));
+  if (N == 0) {  // an empty block contributes nothing to the totals
+    FK_CUDA(cudaMemsetAsync(sums, 0, (size_t)B * K * d * sizeof(float), s));
+    FK_CUDA(cudaMemsetAsync(counts, 0, (size_t)B * K * sizeof(int32_t), s));
+    return FK_OK;
+  }
+  FK_TRY(check_dev(ids, "ids"));
   FK_TRY(check_dev_opt(xn, "xn"));
   const fk_options o = options_of(opts);
   Workspace *ws;

@@ -41,7 +41,7 @@ class CudaSteps:
 
     def point_norms(self, x):
         # fp16 / bf16 points resident on the device: ||x||^2 once per run
-        if x.dtype == torch.float32 or not x.is_cuda:
+        if x.dtype == torch.float32 or not x.is_cuda or x.shape[1] == 0:
             return None
         xn = torch.empty(x.shape[:2], dtype=torch.float32, device=x.device)
         return self._norms(x, xn, stream=self.stream)

@@ -222,7 +222,10 @@ int fk_init_centers(const void *init, int B, int K, int d, int dtype, float *cen
  * (step a1, as fk_assign), then the sort-inverse reduction of the block
  * without the division (steps a2-a5): sums[b,k,:] = sum of the block's points
  * with id k (fp32), counts[b,k] = their number; an empty cluster gets zeros.
- *   shape       the block: N = this rank's points per batch.
+ *   shape       the block: N = this rank's points per batch.  N may be
+ *               below K (clusters without points in the block get zeros)
+ *               or 0 (an empty block: zero sums and counts; x, xn and ids
+ *               are not read and may be NULL).
  *   x           (B, N, d) in dtype: device memory, or pinned host memory
  *               (then streamed in chunks of opts->chunk_points, double-
  *               buffered, as fk_lloyd's streamed mode).

@@ -106,8 +106,15 @@ def test_data_parallel_pieces_validate_on_the_host():
     assert "shape is NULL" in fk.fk_last_error()
     assert L.fk_lloyd_step_partial(ctypes.byref(shape), p, None, p, p, None, p, None, None) == fk.FK_EINVAL
     assert "sums is NULL" in fk.fk_last_error()
-    bad = fk.FkShape(1, 10, 11, 8, fk.FK_F16)
-    assert L.fk_lloyd_step_partial(ctypes.byref(bad), p, None, p, p, p, p, None, None) == fk.FK_EINVAL
+    for bad in (fk.FkShape(1, -1, 4, 8, fk.FK_F16), fk.FkShape(1, 10, 4, 12, fk.FK_F16),
+                fk.FkShape(0, 10, 4, 8, fk.FK_F16)):
+        assert L.fk_lloyd_step_partial(ctypes.byref(bad), p, None, p, p, p, p, None, None) == fk.FK_EINVAL
+    # a block may hold fewer points than clusters, or none: the shape passes and
+    # the first failure is a pointer check (none of these fakes is device memory)
+    for block in (fk.FkShape(1, 10, 11, 8, fk.FK_F16), fk.FkShape(1, 0, 4, 8, fk.FK_F16)):
+        assert L.fk_lloyd_step_partial(ctypes.byref(block), None, None, p, None, p, p, None,
+                                       None) == fk.FK_EINVAL
+        assert "must be device memory" in fk.fk_last_error() or "is NULL" in fk.fk_last_error()
     assert L.fk_update_finalize(p, None, 1, 4, 8, fk.FK_F16, p, p, None, None) == fk.FK_EINVAL
     assert "counts is NULL" in fk.fk_last_error()
     assert L.fk_update_finalize(p, p, 1, 4, 8, 9, p, p, None, None) == fk.FK_EINVAL

@@ -72,6 +72,45 @@ def test_partial_blocks_sum_to_the_update(dtype, d):
         assert torch.equal(cdt, centers.to(TORCH_DT[dtype]))
 
 
+@pytest.mark.parametrize("dtype,d", [("f16", 128), ("f32", 32)])
+def test_blocks_below_k_and_an_empty_block(dtype, d):
+    """Blocks of fewer points than clusters, and an empty block, still add up
+    to the whole update: only the whole problem needs K <= N.  Every output of
+    the partial step is written (the buffers start as 7s), an empty cluster of
+    a block gets zeros and the empty block contributes zero sums and counts."""
+    import clustering_flashassign_b200 as fk
+    from clustering_flashassign_b200.dist import block_of
+    B, N, K, world = 2, 600, 300, 5      # blocks of 120 points, K = 300
+    x, _, c = case(B, N, K, d, dtype, seed=47)
+    xd, cd = to_dev(x, dtype), to_dev(c, dtype)
+    full = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    fk.fk_assign(xd, cd, full)
+    ids_parts, sums, counts = [], None, None
+    for n0, n1 in [block_of(N, r, world) for r in range(world)] + [(N, N)]:
+        xb = xd[:, n0:n1].contiguous()
+        ids_r = torch.empty((B, n1 - n0), dtype=torch.int32, device="cuda")
+        s_r = torch.full((B, K, d), 7.0, dtype=torch.float32, device="cuda")
+        c_r = torch.full((B, K), 7, dtype=torch.int32, device="cuda")
+        fk.fk_lloyd_step_partial(xb, None, cd, ids_r, s_r, c_r)
+        if n1 == n0:
+            torch.cuda.synchronize()
+            assert int(c_r.abs().sum()) == 0 and float(s_r.abs().sum()) == 0.0
+        ids_parts.append(ids_r)
+        sums = s_r if sums is None else sums + s_r
+        counts = c_r if counts is None else counts + c_r
+    ids = torch.cat(ids_parts, dim=1)
+    assert torch.equal(ids, full)
+    centers = torch.empty((B, K, d), dtype=torch.float32, device="cuda")
+    fk.fk_init_centers(cd, centers)
+    cdt = torch.empty_like(cd) if dtype != "f32" else None
+    fk.fk_update_finalize(sums, counts, centers, cdt, dtype=TORCH_DT[dtype])
+    torch.cuda.synchronize()
+    assert fk.fk_device_error() == 0
+    new, rc, _, _ = oracle.update(x, dtype, ids.cpu().numpy(), synthdata.to_f64(c, dtype))
+    np.testing.assert_array_equal(counts.cpu().numpy(), rc)
+    check_centers(centers.cpu().numpy(), new, dtype)
+
+
 def _fk_lloyd(xd, cd, iters, **kw):
     import clustering_flashassign_b200 as fk
     B, N, _ = xd.shape
