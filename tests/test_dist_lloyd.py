@@ -32,6 +32,10 @@ class OracleSteps:
     def partial(self, x, xn, centers_dt, ids, sums, counts):
         xb = x.numpy()
         B, n, d = xb.shape
+        if n == 0:  # an empty block contributes zero totals (as fk_lloyd_step_partial)
+            sums.zero_()
+            counts.zero_()
+            return
         g, _, _ = oracle.assign(xb, "f32", centers_dt.to(torch.float64).numpy())
         ids.copy_(torch.from_numpy(g))
         K = sums.shape[1]
@@ -108,6 +112,7 @@ def test_block_of_covers_every_point_once():
 @pytest.mark.parametrize("world,case", [
     (2, (3, 2, 1001, 9, 4, 6, 0.0)),     # fixed count, uneven blocks, an empty cluster
     (3, (4, 1, 900, 6, 3, 50, 1e-9)),    # tol stop: every rank stops at the same iteration
+    (4, (5, 1, 3, 2, 3, 3, 0.0)),        # more ranks than points: blocks below K, one empty block
 ])
 def test_data_parallel_matches_single_process_lloyd(world, case):
     seed, B, N, K, d, max_iter, tol = case
