@@ -30,6 +30,43 @@ def block_of(N: int, rank: int, world: int) -> tuple[int, int]:
     return n0, n0 + base + (1 if rank < extra else 0)
 
 
+def initial_centers_over_blocks(x: torch.Tensor, K: int, seed: int = 0, group=None) -> torch.Tensor:
+    """The initial centroids of a problem split into contiguous blocks, on every rank.
+
+    x is this rank's block (B, n, d); the blocks in rank order make up the whole
+    problem of N = (sum of n) points per batch.  Returns (B, K, d) in x's dtype on
+    x's device: the points at init_indices(B, N, K, seed) of the whole problem,
+    the centroids a single process with all the points would start from.  Every
+    rank takes the same collective steps: one all-gather of the block sizes, one
+    all-reduce that assembles the rows, each owned by exactly one rank (summed
+    as integer bits with zeros, so every value arrives exactly).
+    """
+    from .kmeans import init_indices
+    B, n, d = x.shape
+    group_rank = dist.get_rank(group)
+    world = dist.get_world_size(group)
+    on_gpu = dist.get_backend(group) == "nccl"
+    cdev = torch.device("cuda", torch.cuda.current_device()) if on_gpu else torch.device("cpu")
+    size = torch.tensor([n], dtype=torch.int64, device=cdev)
+    sizes = [torch.empty_like(size) for _ in range(world)]
+    dist.all_gather(sizes, size, group=group)
+    sizes = [int(t.item()) for t in sizes]
+    N, n0 = sum(sizes), sum(sizes[:group_rank])
+    if K > N:  # every rank knows N now, so every rank raises
+        raise ValueError(f"K = {K} clusters but only {N} points over the ranks")
+    idx = init_indices(B, N, K, seed)
+    rows = torch.zeros((B, K, d), dtype=x.dtype)
+    for b in range(B):
+        mine = ((idx[b] >= n0) & (idx[b] < n0 + n)).nonzero().flatten()
+        if mine.numel():
+            rows[b, mine] = x[b].index_select(0, (idx[b, mine] - n0).to(x.device)).cpu()
+    words = rows.view(torch.int32) if x.element_size() == 4 or d % 2 == 0 else rows.to(torch.float32)
+    words = words.to(cdev)
+    dist.all_reduce(words, op=dist.ReduceOp.SUM, group=group)
+    out = words.view(x.dtype) if words.dtype == torch.int32 else words.to(x.dtype)
+    return out.to(x.device).contiguous()
+
+
 class CudaSteps:
     """The per-rank steps of lloyd_data_parallel, each one call into libfk."""
 

@@ -73,9 +73,11 @@ class FlashKMeans:
       predict(data)      ids against the trained centroids (fk_assign)
       fit_predict(data)  train, then the ids of the last assignment
     device None: the current CUDA device.  When a torch.distributed process group
-    is initialised, every rank passes its own contiguous block of the points and the
-    ranks fit one model together (clustering_flashassign_b200.dist); predict and
-    fit_predict then return the labels of the caller's block.
+    is initialised, every rank passes its own contiguous block of the points (the
+    blocks in rank order make up the data) and the ranks fit one model together
+    (clustering_flashassign_b200.dist), starting from the centroids one process
+    with all the points would pick; predict and fit_predict then return the
+    labels of the caller's block.
     """
 
     def __init__(self, d: int, k: int, niter: int = 20, tol: float = 0.0,
@@ -106,12 +108,9 @@ class FlashKMeans:
         x, squeeze = self._prep(data)
         B, n, d = x.shape
         if dist.is_available() and dist.is_initialized():
-            from .dist import lloyd_data_parallel
-            # every rank draws the initial centroids from rank 0's block, then shares them
-            init = torch.empty((B, self.k, d), dtype=self.dtype, device=self.device)
-            if dist.get_rank() == 0:
-                init.copy_(_initial_centers(x, self.k, self.seed, self.device))
-            dist.broadcast(init, src=0)
+            from .dist import initial_centers_over_blocks, lloyd_data_parallel
+            # the whole problem's initial centroids, assembled from the ranks' blocks
+            init = initial_centers_over_blocks(x, self.k, self.seed).to(self.device)
             xb = x if x.is_cuda or x.is_pinned() else x.to(self.device)
             ids = torch.empty((B, n), dtype=torch.int32, device=self.device)
             centers = torch.empty((B, self.k, d), dtype=torch.float32, device=self.device)

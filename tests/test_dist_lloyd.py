@@ -132,3 +132,48 @@ def test_data_parallel_matches_single_process_lloyd(world, case):
     # the far initial centroid kept its value (its cluster is empty)
     assert (ref["counts"][:, K - 1] == 0).all()
     np.testing.assert_array_equal(res[0][4][:, K - 1], init[:, K - 1].astype(np.float64))
+
+
+def _x_for_init(seed, B, N, d, dtype):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn((B, N, d), generator=g).to(dtype)
+    x[:, :, 0] = -0.0  # a sum with zeros in floating point would turn these into +0.0
+    return x
+
+
+def _init_worker(rank, world, port, case, out):
+    from clustering_flashassign_b200.dist import initial_centers_over_blocks
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        seed, B, N, K, d, dtype = case
+        x = _x_for_init(seed, B, N, d, dtype)
+        n0, n1 = block_of(N, rank, world)
+        got = initial_centers_over_blocks(x[:, n0:n1].contiguous(), K, seed)
+        out[rank] = (str(got.dtype), tuple(got.shape), got.view(torch.int16 if got.element_size() == 2
+                                                                 else torch.int32).numpy().copy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,case", [
+    (2, (7, 2, 1001, 9, 8, torch.float16)),
+    (3, (8, 1, 900, 50, 3, torch.float32)),
+    (4, (9, 2, 3, 2, 8, torch.bfloat16)),   # more ranks than points: blocks below K, an empty block
+])
+def test_initial_centers_over_blocks_are_one_process_choice(world, case):
+    """Every rank gets, bit for bit, the initial centroids a single process with
+    all the points picks (the facade's data-parallel training starts there)."""
+    from clustering_flashassign_b200.kmeans import _initial_centers
+    seed, B, N, K, d, dtype = case
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_init_worker, args=(world, port, case, out), nprocs=world, join=True)
+        res = dict(out)
+    ref = _initial_centers(_x_for_init(seed, B, N, d, dtype), K, seed, "cpu")
+    bits = ref.view(torch.int16 if ref.element_size() == 2 else torch.int32).numpy()
+    for r in range(world):
+        assert res[r][0] == str(ref.dtype) and res[r][1] == tuple(ref.shape)
+        np.testing.assert_array_equal(res[r][2], bits)
