@@ -177,3 +177,30 @@ def test_initial_centers_over_blocks_are_one_process_choice(world, case):
     for r in range(world):
         assert res[r][0] == str(ref.dtype) and res[r][1] == tuple(ref.shape)
         np.testing.assert_array_equal(res[r][2], bits)
+
+
+def _too_few_worker(rank, world, port, out):
+    from clustering_flashassign_b200.dist import initial_centers_over_blocks
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
+    try:
+        try:
+            initial_centers_over_blocks(torch.zeros((1, 2, 4)), 5)   # 2 points per rank, K = 5
+            out[rank] = "returned"
+        except ValueError as e:
+            out[rank] = str(e)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_initial_centers_over_blocks_fail_on_every_rank_together():
+    """K above the whole problem's point count raises on every rank after the
+    size exchange, so no rank is left waiting in a collective."""
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_too_few_worker, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    assert set(res) == {0, 1}
+    assert all("only 4 points" in v for v in res.values()), res
