@@ -152,9 +152,22 @@ def fk_assign(x: torch.Tensor, c: torch.Tensor, ids: torch.Tensor, stream=None) 
 
 
 def fk_assign_noalloc(x: torch.Tensor, c: torch.Tensor, ids: torch.Tensor, stream=None) -> torch.Tensor:
-    """fk_assign that allocates no device memory (static scratch; see include/fk.h)."""
+    """fk_assign that allocates no device memory (static scratch; see include/fk.h).
+
+    The C entry point makes no pointer query (so that it can run where the
+    runtime refuses one), so the placement of the tensors is checked here:
+    all three on one CUDA device, ids int32 of shape (B, N)."""
     B, N, d = x.shape
     K = c.shape[1]
+    for name, t in (("x", x), ("c", c), ("ids", ids)):
+        if not t.is_cuda:
+            raise ValueError(f"fk_assign_noalloc: {name} must be a CUDA tensor")
+        if t.device != x.device:
+            raise ValueError(f"fk_assign_noalloc: {name} is on {t.device}, x on {x.device}")
+    if ids.dtype != torch.int32 or tuple(ids.shape) != (B, N):
+        raise ValueError(f"fk_assign_noalloc: ids must be int32 of shape {(B, N)}")
+    if c.dtype != x.dtype or c.dim() != 3 or c.shape[0] != B or c.shape[2] != d:
+        raise ValueError("fk_assign_noalloc: c must be (B, K, d) in x's dtype")
     with _on(x, c, ids):
         _check(lib.fk_assign_noalloc(_ptr(x), _ptr(c), B, N, K, d, _dtype_code(x), _ptr(ids),
                                      _stream(stream)), "fk_assign_noalloc")

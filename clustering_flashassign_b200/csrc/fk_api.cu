@@ -7,6 +7,20 @@
 #include "fk_internal.h"
 
 namespace fk {
+
+int check_shape(int B, long long N, int K, int d, int dtype) {
+  if (dtype != FK_F32 && dtype != FK_F16 && dtype != FK_BF16)
+    return set_error(FK_EINVAL, "unknown dtype " + std::to_string(dtype));
+  if (B <= 0 || N <= 0 || K <= 0 || d <= 0) return set_error(FK_EINVAL, "B, N, K and d must be positive");
+  if (N > 0x7fffffffLL) return set_error(FK_EINVAL, "N must be below 2^31");
+  if ((long long)K > N) return set_error(FK_EINVAL, "K must not exceed N");
+  if (B > 65535) return set_error(FK_EUNSUPPORTED, "B above 65535");
+  if (K > (1 << 24)) return set_error(FK_EUNSUPPORTED, "K above 2^24");
+  if (dtype != FK_F32 && (d * 2) % 16 != 0)
+    return set_error(FK_EINVAL, "fp16/bf16 rows must be a multiple of 16 bytes (d % 8 == 0)");
+  return FK_OK;
+}
+
 namespace {
 
 enum Loc { LOC_DEVICE, LOC_HOST_PINNED, LOC_HOST_PAGEABLE };
@@ -20,19 +34,6 @@ Loc locate(const void *p) {
   if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) return LOC_DEVICE;
   if (at.type == cudaMemoryTypeHost) return LOC_HOST_PINNED;
   return LOC_HOST_PAGEABLE;
-}
-
-int check_shape(int B, long long N, int K, int d, int dtype) {
-  if (dtype != FK_F32 && dtype != FK_F16 && dtype != FK_BF16)
-    return set_error(FK_EINVAL, "unknown dtype " + std::to_string(dtype));
-  if (B <= 0 || N <= 0 || K <= 0 || d <= 0) return set_error(FK_EINVAL, "B, N, K and d must be positive");
-  if (N > 0x7fffffffLL) return set_error(FK_EINVAL, "N must be below 2^31");
-  if ((long long)K > N) return set_error(FK_EINVAL, "K must not exceed N");
-  if (B > 65535) return set_error(FK_EUNSUPPORTED, "B above 65535");
-  if (K > (1 << 24)) return set_error(FK_EUNSUPPORTED, "K above 2^24");
-  if (dtype != FK_F32 && (d * 2) % 16 != 0)
-    return set_error(FK_EINVAL, "fp16/bf16 rows must be a multiple of 16 bytes (d % 8 == 0)");
-  return FK_OK;
 }
 
 // Options with the environment's defaults: FK_VERBOSE=1 turns the per-iteration

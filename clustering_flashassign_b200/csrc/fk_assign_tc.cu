@@ -34,7 +34,13 @@
 //               per value) and keeps a three-input float max (half an
 //               instruction per value).  Columns whose acc agree in all other
 //               bits count as tied and the lowest column wins; that merges
-//               values within 2^-15 of each other (relative).
+//               values within 2^-15 of each other (relative).  Relative to
+//               |acc| that is harmless while the nearest squared distance is
+//               below 16 ||x||^2 (the merged values then lie within 5e-4 ||x||^2
+//               of each other).  A point beyond that bound (far from every
+//               centroid compared with its own norm, e.g. x = 0) is flagged at
+//               the end of its tile and re-ranked exactly: one warp computes
+//               sum_j (x_j - c_kj)^2 in fp64 for every k (lowest k on ties).
 //   split-d     (d > 128): each pipeline stage carries a 64-wide slice of the
 //               point tile and the matching centroid slice; the d loop runs
 //               inside each K chunk (the pages' split-D path, "flash-kmeans
@@ -54,8 +60,7 @@
 // columns carry a sentinel norm row (acc about -2^31 or below) so they never win.
 #include <cuda.h>
 
-#include "fk_norms.cuh"
-#include "fk_sm100.cuh"
+#include "fk_assign_common.cuh"
 
 namespace fk {
 namespace {
@@ -71,7 +76,6 @@ constexpr uint32_t kAExtBytes = kTileM * kExt * 2;        // 4 KB of point norm 
 constexpr uint32_t kBExtBytes = kChunkN * kExt * 2;       // 8 KB of centroid norm rows
 constexpr int kExtSlots = 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kKeyMask = 0xFFFFFF00u;  // packed keys: column in the low byte
 
 struct TcArgs {
   int N;
@@ -87,6 +91,11 @@ struct TcArgs {
   // optional: the counting sort's tile histogram, H[b][row / 2048][id] += 1
   uint32_t *hist;
   int hist_tiles;
+  // resident variant: the points and centroids in global memory (B, N, d) and
+  // (B, K, d), read only by the exact re-rank of flagged points
+  const void *xg;
+  const void *cg;
+  int d;
   // split-d only, optional: per-point packed (value, index) keys; then every
   // (tile, chunk) pair is its own work item and chunks merge by atomicMax
   unsigned long long *keys;
@@ -116,11 +125,15 @@ struct Layout {
       RESIDENT ? KB * kCBlockBytes + kBExtBytes : kXBlockBytes + kCBlockBytes;
   static constexpr uint32_t kBarOff = kStagesOff + STAGES * kStageBytes;
   // barriers: full[S], empty[S], efull[E], eempty[E], xfull[2], xempty[2],
-  //           xnfull[2], accfull[2], accempty[2], mfull[2], mempty[2], drain
-  static constexpr int kNumBars = 2 * STAGES + 2 * kExtSlots + 15;
+  //           xnfull[2], accfull[2], accempty[2], mfull[2], mempty[2], drain,
+  //           xnfree[2]
+  static constexpr int kNumBars = 2 * STAGES + 2 * kExtSlots + 17;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag
   static constexpr uint32_t kMergeOff = (kMiscOff + 16 + 15) / 16 * 16;
-  static constexpr uint32_t kBytes = kMergeOff + 2 * kTileM * 8;
+  // resident: ||x||^2 of the rows of the two point-tile buffers, for the
+  // epilogue's far-point check
+  static constexpr uint32_t kXnOff = kMergeOff + 2 * kTileM * 8;
+  static constexpr uint32_t kBytes = kXnOff + (RESIDENT ? 2 * kTileM * 4 : 0);
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
   static_assert(kStagesOff % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
@@ -146,90 +159,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   r = __shfl_sync(0xffffffffu, r, 0);
   __syncwarp();
   return r != 0;
-}
-
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-__device__ __forceinline__ float key_hi(float key) {
-  return __uint_as_float(__float_as_uint(key) & kKeyMask);
-}
-
-// One MMA step of the element type's kind: kind::f16 for fp16 / bf16 (K = 16),
-// kind::tf32 for fp32 (K = 8); either way 32 bytes of every operand row.
-template <typename T>
-__device__ __forceinline__ void mma_t(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                      uint32_t accumulate) {
-  if constexpr (sizeof(T) == 4) mma_tf32(d_tmem, a_desc, b_desc, idesc, accumulate);
-  else mma_f16(d_tmem, a_desc, b_desc, idesc, accumulate);
-}
-
-// Stores one 32-byte norm row at row r of a K-major 32-byte-swizzled tile:
-// 16-byte chunk q of row r sits at r * 32 + ((q ^ ((r >> 2) & 1)) * 16).
-__device__ __forceinline__ void store_row32_sw32(uint8_t *tile, int r, const void *row) {
-  const int flip = (r >> 2) & 1;
-  uint4 *p = reinterpret_cast<uint4 *>(tile + r * 32);
-  p[flip] = reinterpret_cast<const uint4 *>(row)[0];
-  p[flip ^ 1] = reinterpret_cast<const uint4 *>(row)[1];
-}
-template <typename T>
-__device__ __forceinline__ void store_ext_row_sw32(uint8_t *tile, int r, const T (&row)[kExt]) {
-  store_row32_sw32(tile, r, row);
-}
-
-// a0 += lo(v)^2, a1 += hi(v)^2 for two packed 16-bit values, fp32 accumulation
-// (mixed-precision FMA: the 16-bit inputs are exact in fp32, one rounding).
-template <typename T> __device__ __forceinline__ void sq2_acc(uint32_t v, float &a0, float &a1);
-template <> __device__ __forceinline__ void sq2_acc<__half>(uint32_t v, float &a0, float &a1) {
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-      "fma.rn.f32.f16 %0, lo, lo, %0;\n\tfma.rn.f32.f16 %1, hi, hi, %1;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "r"(v));
-}
-template <> __device__ __forceinline__ void sq2_acc<__nv_bfloat16>(uint32_t v, float &a0, float &a1) {
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-      "fma.rn.f32.bf16 %0, lo, lo, %0;\n\tfma.rn.f32.bf16 %1, hi, hi, %1;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "r"(v));
-}
-
-// Running argmax over one 32-column TMEM load with packed keys: the low byte
-// of each (negative) accumulator is replaced by its column (a byte taken from
-// colb, which holds the bytes 0..127).  For negative floats a larger key means
-// a smaller |acc|, and among equal upper bits the smaller column.  Four
-// independent max chains.
-__device__ __forceinline__ void scan_packed(const uint32_t (&r)[32], const uint32_t cb,
-                                            const uint32_t (&colb)[32], float &m0, float &m1,
-                                            float &m2, float &m3) {
-#define FK_KEY(t) __uint_as_float(__byte_perm(r[j + (t)], colb[(cb + j + (t)) >> 2], 0x3214u + ((cb + j + (t)) & 3u)))
-#pragma unroll
-  for (int j = 0; j < 32; j += 8) {
-    m0 = max3f(m0, FK_KEY(0), FK_KEY(1));
-    m1 = max3f(m1, FK_KEY(2), FK_KEY(3));
-    m2 = max3f(m2, FK_KEY(4), FK_KEY(5));
-    m3 = max3f(m3, FK_KEY(6), FK_KEY(7));
-  }
-#undef FK_KEY
-}
-
-// Exact running argmax over one 32-column TMEM load: chain t sees columns
-// j = t (mod 4) in increasing order and moves only on a strictly larger value.
-__device__ __forceinline__ void scan_exact(const uint32_t (&r)[32], const int cb, float (&lb)[4],
-                                           int (&li)[4]) {
-#pragma unroll
-  for (int j = 0; j < 32; j += 4) {
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const float v = __uint_as_float(r[j + t]);
-      if (v > lb[t]) {
-        lb[t] = v;
-        li[t] = cb + j + t;
-      }
-    }
-  }
 }
 
 template <typename T, bool RESIDENT, int KB, int STAGES>
@@ -260,6 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto mfull = [&](int i) { return bar0 + 8u * (kB2 + 10 + i); };
   auto mempty = [&](int i) { return bar0 + 8u * (kB2 + 12 + i); };
   const uint32_t drain = bar0 + 8u * (kB2 + 14);
+  auto xnfree = [&](int i) { return bar0 + 8u * (kB2 + 15 + i); };
+  float *xnorm_s = reinterpret_cast<float *>(smem + L::kXnOff);  // [2][kTileM], resident only
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   float2 *merge = reinterpret_cast<float2 *>(smem + L::kMergeOff);
@@ -283,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(accempty(i), kEpiWarps);
       mbar_init(mfull(i), kEpiWarps / 2);
       mbar_init(mempty(i), kEpiWarps / 2);
+      mbar_init(xnfree(i), kEpiWarps / 2);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -529,6 +461,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           store_ext_row_sw32<T>(smem + L::kAExtOff + xb * kAExtBytes, q * 32 + lane, row);
         }
         if (clamped) atomicCAS(a.err, DEV_OK, DEV_RANGE);
+        // the norms for the epilogue's far-point check, once the epilogue has
+        // finished the tile that used this buffer before (two tiles back); the
+        // epilogue reads them after xnfull, so tile g + 2 cannot complete xnfull
+        // before tile g's norms are read
+        if (!warp_wait(xnfree(xb), ((g >> 1) & 1) ^ 1, abort_flag, a.err, lane)) break;
+#pragma unroll
+        for (int q = 0; q < kTileM / 32; ++q) xnorm_s[xb * kTileM + q * 32 + lane] = xn2[q];
         fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
         __syncwarp();
         if (lane == 0) mbar_arrive(xnfull(xb));
@@ -637,6 +576,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           idx = oi;
         }
         const int row = row0 + r_in_tile;
+        if constexpr (RESIDENT) {
+          // far-point check (see the header): flagged rows of this warp are
+          // re-ranked one after another by the whole warp
+          // xnfull of this tile completed before its first MMA; waiting on it
+          // here orders the norm warp's stores before these reads
+          if (!warp_wait(xnfull(p), (u >> 1) & 1, abort_flag, a.err, lane)) { ok = false; break; }
+          const float xn = xnorm_s[p * kTileM + r_in_tile];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xnfree(p));  // the norm warp may reuse the slot
+          unsigned flagged = __ballot_sync(0xffffffffu, row < a.N && -val > kFarRatioHalf * xn);
+          while (flagged) {
+            const int src = __ffs(flagged) - 1;
+            flagged &= flagged - 1;
+            const int r = row0 + quad * 32 + src;
+            const T *xrow = static_cast<const T *>(a.xg) + ((size_t)b * a.N + r) * a.d;
+            const T *cb = static_cast<const T *>(a.cg) + (size_t)b * a.K * a.d;
+            const int k = exact_argmin_warp<T>(xrow, cb, a.K, a.d, lane);
+            if (lane == src) idx = k;
+          }
+        }
         if (row < a.N && per_chunk) {  // this chunk's best; the chunks merge in the keys
           atomicMax(a.keys + (size_t)b * a.N + row, pack_argmax(val, idx));
         } else if (row < a.N) {
@@ -810,6 +769,9 @@ int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float
   a.xn = xn;
   a.ids = ids;
   a.err = err;
+  a.xg = x;
+  a.cg = ch;
+  a.d = d;
   a.idesc = sm100::idesc_f32acc(dtype == FK_F32 ? 2u : dtype == FK_BF16 ? 1u : 0u, kTileM, kChunkN);
   // split-d (fp32, or more than two 16-bit K-blocks): with keys, one work item
   // per (tile, chunk) and a merge of the chunks' results

@@ -109,6 +109,12 @@ const char *last_error();
 size_t esize(int dtype);
 int num_sms();
 
+// Shape and dtype rules shared by every entry point that takes (B, N, K, d):
+// FK_EINVAL for an unknown dtype, a size <= 0, N >= 2^31, K > N, or 16-bit
+// rows that are not a multiple of 16 bytes; FK_EUNSUPPORTED for B > 65535 or
+// K > 2^24.
+int check_shape(int B, long long N, int K, int d, int dtype);
+
 // Programmatic dependent launch: the kernels of one Lloyd iteration are
 // launched so that each may start while its predecessor in the stream drains.
 // A kernel launched this way calls pdl_wait() before it reads anything an

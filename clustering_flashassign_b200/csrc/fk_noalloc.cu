@@ -55,14 +55,7 @@ using namespace fk;
 extern "C" int fk_assign_noalloc(const void *x, const void *c, int B, long long N, int K, int d,
                                  int dtype, int32_t *ids, fk_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype != FK_F32 && dtype != FK_F16 && dtype != FK_BF16)
-    return set_error(FK_EINVAL, "unknown dtype " + std::to_string(dtype));
-  if (B <= 0 || N <= 0 || K <= 0 || d <= 0) return set_error(FK_EINVAL, "B, N, K and d must be positive");
-  if (N > 0x7fffffffLL) return set_error(FK_EINVAL, "N must be below 2^31");
-  if ((long long)K > N) return set_error(FK_EINVAL, "K must not exceed N");
-  if (B > 65535) return set_error(FK_EUNSUPPORTED, "B above 65535");
-  if (dtype != FK_F32 && (d * 2) % 16 != 0)
-    return set_error(FK_EINVAL, "fp16/bf16 rows must be a multiple of 16 bytes (d % 8 == 0)");
+  FK_TRY(check_shape(B, N, K, d, dtype));  // the same rules as fk_assign
   if (!x || !c || !ids) return set_error(FK_EINVAL, "x, c and ids must not be NULL");
   const bool tc = dtype != FK_F32;
   if (tc && ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(c)) & 15u))

@@ -1,4 +1,7 @@
-"""Data-parallel Lloyd: the points of every batch split into contiguous blocks, one per rank.
+"""Data-parallel Lloyd over several processes, one GPU each, in two splits.
+
+Point blocks (lloyd_data_parallel): the points of every batch split into
+contiguous blocks, one per rank.
 
 The pages' large-N path splits the N points into contiguous block
 partitions, one per GPU; each GPU runs its own assign and partial update over
@@ -15,6 +18,17 @@ memory or in pinned host memory (then it is streamed in chunks).
 
     n0, n1 = block_of(N, rank, world)
     iters = lloyd_data_parallel(x[:, n0:n1], init, max_iter, tol, ids, centers)
+
+Batch shares (lloyd_batch_split): the B batches of a problem are independent
+K-Means problems, so each rank takes a contiguous share of them and runs the
+whole Lloyd loop on its share with no exchange of data at all; the only
+collective in the loop is a max of one float per iteration when tol > 0 (the
+stop rule is one global max-shift test over every batch), and the results
+are gathered once at the end (gather_batches).
+
+    b0, b1 = block_of(B, rank, world)
+    iters = lloyd_batch_split(x[b0:b1], init[b0:b1], max_iter, tol, ids_share, centers_share)
+    ids_all = gather_batches(ids_share, B)
 """
 from __future__ import annotations
 
@@ -68,7 +82,7 @@ def initial_centers_over_blocks(x: torch.Tensor, K: int, seed: int = 0, group=No
 
 
 class CudaSteps:
-    """The per-rank steps of lloyd_data_parallel, each one call into libfk."""
+    """The per-rank steps of lloyd_data_parallel and lloyd_batch_split, each one call into libfk."""
 
     def __init__(self, stream=None, chunk_points: int = 0):
         from . import fk_init_centers, fk_lloyd_step_partial, fk_point_norms, fk_update_finalize
@@ -137,3 +151,60 @@ def lloyd_data_parallel(x: torch.Tensor, init_centers: torch.Tensor, max_iter: i
         if tol > 0 and float(shift.item()) < tol:
             break
     return it
+
+
+def lloyd_batch_split(x: torch.Tensor, init_centers: torch.Tensor, max_iter: int, tol: float,
+                      ids: torch.Tensor, centers: torch.Tensor, group=None, steps=None) -> int:
+    """Lloyd's iterations over this rank's share of the batches.
+
+    x             (b, N, d): this rank's contiguous share of the batches (b may be 0).
+    init_centers  (b, K, d) in x's dtype: their initial centroids.
+    ids, centers  (b, N) int32 and (b, K, d) out.
+    The batches never exchange data.  With tol > 0 the ranks agree on the stop:
+    after every iteration one all-reduce takes the max of the ranks' max shifts,
+    so every rank stops after the iteration a single process over all the
+    batches would stop after.  With tol <= 0 the loop takes no collective step.
+    Returns the number of iterations run.
+    """
+    steps = steps or CudaSteps()
+    b, _, d = x.shape
+    K = init_centers.shape[1]
+    dev = centers.device
+    agree = tol > 0 and dist.is_available() and dist.is_initialized()
+    shift = torch.zeros((1,), dtype=centers.dtype, device=dev)
+    if b > 0:
+        sums = torch.empty((b, K, d), dtype=centers.dtype, device=dev)
+        counts = torch.empty((b, K), dtype=torch.int32, device=dev)
+        steps.init_centers(init_centers, centers)
+    low = x.dtype in (torch.float16, torch.bfloat16)
+    centers_dt = torch.empty_like(init_centers) if low else None
+    cur = init_centers if low else centers
+    xn = steps.point_norms(x) if b > 0 else None
+    it = 0
+    while it < max_iter:
+        if b > 0:
+            steps.partial(x, xn, cur, ids, sums, counts)
+            steps.finalize(sums, counts, centers, centers_dt, shift, x.dtype)
+        it += 1
+        if low:
+            cur = centers_dt
+        if tol > 0:
+            if agree:
+                dist.all_reduce(shift, op=dist.ReduceOp.MAX, group=group)
+            if float(shift.item()) < tol:
+                break
+    return it
+
+
+def gather_batches(share: torch.Tensor, B: int, group=None) -> torch.Tensor:
+    """The (B, ...) tensor whose batches [b0, b1) are each rank's `share`
+    (block_of(B, rank, world)), on every rank: one all-gather of the shares
+    padded to the largest one."""
+    world = dist.get_world_size(group)
+    per = -(-B // world)
+    pad = torch.zeros((per,) + tuple(share.shape[1:]), dtype=share.dtype, device=share.device)
+    pad[: share.shape[0]] = share
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    out = [parts[r][: block_of(B, r, world)[1] - block_of(B, r, world)[0]] for r in range(world)]
+    return torch.cat(out, dim=0)

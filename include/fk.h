@@ -258,7 +258,14 @@ int fk_update_finalize(const float *sums, const int32_t *counts, int B, int K, i
 /*
  * fk_assign_noalloc -- fk_assign for callers that cannot allocate device
  * memory (no counterpart in the paper; it is an interface addition).
- * Same arguments, layouts and result as fk_assign.  Callers that run under an
+ * Same arguments, layouts and shape rules as fk_assign.  fp16 / bf16 run the
+ * same kernel as fk_assign and return the same ids.  fp32 always runs the
+ * CUDA-core kernel here (sum_j (x_j - c_j)^2 directly), while fk_assign moves
+ * fp32 problems with d % 4 == 0 and K * d >= 16384 to the 3xTF32 tensor-core
+ * path, whose scratch (a widened copy of the points) this call cannot hold;
+ * on those shapes the two calls may pick different ids for points whose two
+ * nearest centroids lie within 1e-3 ||x||^2 of each other (a near tie), and
+ * this call is much slower.  Callers that run under an
  * allocator owning all device memory, or in loops where allocation (and the
  * synchronization a cudaFree can bring) is not allowed, cannot let fk_assign
  * grow its workspace; this call allocates nothing.  Its scratch (the
@@ -276,8 +283,13 @@ int fk_update_finalize(const float *sums, const int32_t *counts, int B, int K, i
  *   before any stream capture.
  *   All calls on a device share the array: calls that overlap on the GPU
  *   (e.g. on two streams) race and may return wrong ids.  The error word is
- *   cleared at the start of each call; a bounded-wait timeout inside this
- *   variant is recorded there and is not reported by fk_device_error().
+ *   cleared at the start of each call.  What the kernels record there is
+ *   not reported by fk_device_error(), nor by this call (which does not
+ *   synchronize): a bounded-wait timeout, and an fp16 squared norm of 2^32
+ *   or more (a centroid or point with ||v|| >= 65536), where fk_assign
+ *   reports FK_EUNSUPPORTED and this call returns unreliable ids.  Callers
+ *   whose fp16 data may reach that range use fk_assign, or bf16 (whose norm
+ *   digits have the fp32 range).
  */
 int fk_assign_noalloc(const void *x, const void *c, int B, long long N, int K, int d, int dtype,
                       int32_t *ids, fk_stream_t stream);

@@ -159,3 +159,38 @@ def test_binding_runs_each_call_on_its_first_cuda_tensors_device(monkeypatch):
     with fk._on(Tensor(None), None):
         pass
     assert seen == ["cuda:1"]
+
+
+def test_noalloc_binding_rejects_host_tensors_before_any_launch(monkeypatch):
+    """fk_assign_noalloc's C entry point makes no pointer query, so the binding
+    checks the tensors' placement itself: host tensors, or ids of the wrong
+    type or shape, raise ValueError and the library is never called."""
+    import torch
+    import clustering_flashassign_b200 as fk
+
+    calls = []
+
+    class Lib:
+        def __getattr__(self, name):
+            calls.append(name)
+            raise AssertionError(f"library called: {name}")
+
+    monkeypatch.setattr(fk, "lib", Lib())
+    x = torch.zeros(1, 16, 8, dtype=torch.float16)
+    c = torch.zeros(1, 4, 8, dtype=torch.float16)
+    ids = torch.zeros(1, 16, dtype=torch.int32)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        fk.fk_assign_noalloc(x, c, ids)
+    assert calls == []
+    assert fk.FK_OK == 0  # the module itself is intact
+
+
+def test_noalloc_entry_point_shares_fk_assign_shape_rules():
+    import clustering_flashassign_b200 as fk
+    L = fk.lib
+    d = ctypes.c_void_p(0x1000)
+    for B, N, K, dd, dt in [(1, 10, 11, 8, 1), (1, 10, 2, 12, 1), (1, 10, 2, 8, 7), (0, 10, 2, 8, 1)]:
+        assert L.fk_assign_noalloc(d, d, B, N, K, dd, dt, d, None) == fk.FK_EINVAL
+    # K above 2^24 is refused by both (fp32 needs no scratch, so only the shape rule applies)
+    assert L.fk_assign(d, d, 1, 1 << 26, (1 << 24) + 1, 8, fk.FK_F32, d, None) == fk.FK_EUNSUPPORTED
+    assert L.fk_assign_noalloc(d, d, 1, 1 << 26, (1 << 24) + 1, 8, fk.FK_F32, d, None) == fk.FK_EUNSUPPORTED

@@ -179,3 +179,25 @@ def test_nccl_group_of_one_rank():
         assert torch.equal(cen_a, cen_b)
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("dtype,d", [("f16", 128), ("bf16", 256), ("f32", 32)])
+def test_batch_shares_are_fk_lloyd_on_all_batches(dtype, d):
+    """lloyd_batch_split over the shares of three ranks, run one after another
+    in this process (no exchange is needed with tol = 0), concatenates to
+    fk_lloyd over all the batches bit for bit: the batches never interact."""
+    from clustering_flashassign_b200.dist import block_of, lloyd_batch_split
+    B, N, K, world = 5, 1500, 120, 3
+    x, _, c = case(B, N, K, d, dtype, seed=47)
+    xd, cd = to_dev(x, dtype), to_dev(c, dtype)
+    ids_a, cen_a = _fk_lloyd(xd, cd, 3)
+    ids_b, cen_b = [], []
+    for r in range(world):
+        b0, b1 = block_of(B, r, world)
+        ids = torch.empty((b1 - b0, N), dtype=torch.int32, device="cuda")
+        cen = torch.empty((b1 - b0, K, d), dtype=torch.float32, device="cuda")
+        assert lloyd_batch_split(xd[b0:b1].contiguous(), cd[b0:b1].contiguous(), 3, 0.0, ids, cen) == 3
+        ids_b.append(ids)
+        cen_b.append(cen)
+    assert torch.equal(ids_a, torch.cat(ids_b))
+    assert torch.equal(cen_a, torch.cat(cen_b))

@@ -17,7 +17,7 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import oracle
-from clustering_flashassign_b200.dist import block_of, lloyd_data_parallel
+from clustering_flashassign_b200.dist import block_of, gather_batches, lloyd_batch_split, lloyd_data_parallel
 
 
 class OracleSteps:
@@ -204,3 +204,48 @@ def test_initial_centers_over_blocks_fail_on_every_rank_together():
         res = dict(out)
     assert set(res) == {0, 1}
     assert all("only 4 points" in v for v in res.values()), res
+
+
+def _split_worker(rank, world, port, case, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        seed, B, N, K, d, max_iter, tol = case
+        x, init = _data(seed, B, N, K, d)
+        b0, b1 = block_of(B, rank, world)
+        xs = torch.from_numpy(np.ascontiguousarray(x[b0:b1]))
+        ids = torch.empty((b1 - b0, N), dtype=torch.int32)
+        centers = torch.empty((b1 - b0, K, d), dtype=torch.float64)
+        it = lloyd_batch_split(xs, torch.from_numpy(np.ascontiguousarray(init[b0:b1])), max_iter, tol, ids,
+                               centers, steps=OracleSteps())
+        all_ids = gather_batches(ids, B)
+        all_c = gather_batches(centers, B)
+        out[rank] = (it, all_ids.numpy().copy(), all_c.numpy().copy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,case", [
+    (2, (6, 5, 400, 7, 4, 5, 0.0)),      # fixed count, 3 + 2 batches
+    (3, (7, 4, 300, 5, 3, 60, 1e-9)),    # tol stop decided over all batches
+    (3, (8, 2, 200, 4, 2, 4, 0.0)),      # more ranks than batches: one rank holds none
+])
+def test_batch_split_matches_single_process_lloyd(world, case):
+    """Each rank runs its share of the batches; after the gather every rank
+    holds the single-process result, and with tol every rank stopped after the
+    same iteration as the single process (the global max-shift rule)."""
+    seed, B, N, K, d, max_iter, tol = case
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_split_worker, args=(world, port, case, out), nprocs=world, join=True)
+        res = dict(out)
+    x, init = _data(seed, B, N, K, d)
+    ref = oracle.lloyd(x, "f32", init, max_iter, tol, round_dtype=None)
+    assert {res[r][0] for r in range(world)} == {ref["iters"]}
+    if tol > 0:
+        assert ref["iters"] < max_iter, "the tol case should stop early"
+    for r in range(world):
+        np.testing.assert_array_equal(res[r][1], ref["ids"])
+        np.testing.assert_allclose(res[r][2], ref["centers"], rtol=1e-12, atol=1e-12)

@@ -2,8 +2,12 @@
 
 For each shape, fk_lloyd runs all but the last iteration; the last iteration
 then runs step by step through the C ABI so that every output can be checked:
-- ids on a sample of points against the oracle's assign with the GPU's
-  dtype centroids (near-tie rule),
+- every id of the first and the last batch against the oracle's assign with
+  the GPU's dtype centroids (near-tie rule) where that costs the oracle a few
+  seconds (the first batch's tiles are each CTA's first tiles, the last
+  batch's its last ones, so the persistent schedule's tile-ahead buffers and
+  barrier phases are checked over many tiles per CTA), else a random sample
+  of their points; 256 random points of every other batch,
 - counts and perm of the counting sort bit-exact against the oracle,
 - the updated centroids against the oracle's fp64 means of the GPU's ids,
 - and the one-call fk_lloyd result against that stepwise result.
@@ -20,6 +24,7 @@ from test_parity_kernels import to_dev
 pytestmark = pytest.mark.gpu
 
 TORCH_DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+FULL_TERMS = 1.5e11   # a few seconds of the fp64 oracle on the host's cores
 
 
 @pytest.mark.parametrize("name", ["tiny", "api", "zipf", "splitd", "f32large"])
@@ -39,9 +44,17 @@ def test_full_size_workload(name):
     fk.fk_assign(xd, ch, ids)
     g = ids.cpu().numpy()
     rng = np.random.default_rng(17)
-    sample = np.sort(rng.choice(w.N, size=min(w.N, 256), replace=False))
-    xs = np.ascontiguousarray(x[:, sample])
-    check_ids(g[:, sample], xs, w.dtype, chat)
+    ends = sorted({0, w.B - 1})
+    # about FULL_TERMS point-centroid-dimension terms of oracle work per batch
+    n_full = min(w.N, max(4096, int(FULL_TERMS / (w.K * w.d))))
+    for b in ends:
+        pts = np.arange(w.N) if n_full == w.N else np.sort(rng.choice(w.N, size=n_full, replace=False))
+        check_ids(g[b:b + 1, pts], np.ascontiguousarray(x[b:b + 1, pts]), w.dtype, chat[b:b + 1])
+    rest = [b for b in range(w.B) if b not in ends]
+    if rest:
+        sample = np.sort(rng.choice(w.N, size=min(w.N, 256), replace=False))
+        xs = np.ascontiguousarray(x[rest][:, sample])
+        check_ids(g[rest][:, sample], xs, w.dtype, chat[rest])
 
     perm = torch.empty_like(ids)
     counts = torch.empty((w.B, w.K), dtype=torch.int32, device="cuda")

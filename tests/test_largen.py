@@ -3,10 +3,12 @@ copies overlapped with assign / sort / segment reduce, finalize once per
 iteration (the large-N workload: B=1, d=128, K=32768, fp16 mixture of 32768
 components).
 
-By default the workload runs at N = 2^24 (4 GiB of points, 16 chunks of 2^20
-points, so the double-buffered pipeline and the per-chunk accumulation are
-exercised many times).  FK_LARGEN_FULL=1 runs the full N = 2^28 (64 GiB of
-pinned host memory) with the default 2^24-point chunks.
+The workload runs at N = 2^24 in chunks of 2^20 points (4 GiB of points, 16
+chunks, so the double-buffered pipeline and the per-chunk accumulation are
+exercised many times) and at N = 2^25 with the library's default 2^24-point
+chunks (8 GiB: two full 4 GiB chunks alternate the two device buffers, the
+shape of every chunk of the full run).  FK_LARGEN_FULL=1 runs the full
+N = 2^28 (64 GiB of pinned host memory) in place of the 2^25 case.
 
 Lockstep parity after one iteration: sampled ids against the checker's assign
 with the initial centroids; every centroid against the checker's update given
@@ -25,16 +27,17 @@ from parity import check_centers, check_ids
 pytestmark = pytest.mark.gpu
 
 
-def _workload():
+def _workload(points, chunk):
     w = synthdata.WORKLOADS["largen"]
-    if os.environ.get("FK_LARGEN_FULL") == "1":
+    if os.environ.get("FK_LARGEN_FULL") == "1" and chunk == 0:
         return w, 0
-    return synthdata.scaled(w, N=1 << 24), 1 << 20
+    return synthdata.scaled(w, N=points), chunk
 
 
-def test_largen_streamed_from_pinned_host():
+@pytest.mark.parametrize("points,chunk", [(1 << 24, 1 << 20), (1 << 25, 0)])
+def test_largen_streamed_from_pinned_host(points, chunk):
     import clustering_flashassign_b200 as fk
-    w, chunk = _workload()
+    w, chunk = _workload(points, chunk)
     xt = torch.empty((w.B, w.N, w.d), dtype=torch.float16, pin_memory=True)
     x = xt.numpy()
     x_, idx, init = synthdata.make(w, out=x)

@@ -14,7 +14,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synthdata
+from parity import check_ids
 
 pytestmark = pytest.mark.gpu
 
@@ -66,3 +68,24 @@ def test_noalloc_assign_rejects_shapes_beyond_its_scratch():
     st = fk.lib.fk_assign_noalloc(d, d, 5, 300000, 32768, 128, fk.FK_F16, d, None)
     assert st == fk.FK_EUNSUPPORTED
     assert "exceeds" in fk.fk_last_error()
+
+
+def test_noalloc_fp32_on_cuda_cores_matches_the_oracle_where_fk_assign_uses_tf32():
+    """fp32 with K * d >= 16384: fk_assign takes the 3xTF32 tensor-core path,
+    this call the CUDA-core kernel (it cannot hold the widened points).  Both
+    must satisfy the near-tie rule against the fp64 oracle; they may differ
+    from each other only on near ties."""
+    import clustering_flashassign_b200 as fk
+    B, N, K, d = 2, 1500, 300, 64   # K * d = 19200
+    x, c = _inputs(B, N, K, d, "f32", 8)
+    chat = c.cpu().numpy().astype(np.float64)
+    xn = x.cpu().numpy()
+    ref, gap, _ = oracle.assign(xn, "f32", chat)
+    for n in range(2):
+        got = torch.full((B, N), -1, dtype=torch.int32, device="cuda")
+        assert _raw_noalloc(fk, x, c, got) == fk.FK_OK, fk.fk_last_error()
+        torch.cuda.synchronize()
+        check_ids(got.cpu().numpy(), xn, "f32", chat, ref, gap)
+        tc = torch.empty((B, N), dtype=torch.int32, device="cuda")
+        fk.fk_assign(x, c, tc)
+        check_ids(tc.cpu().numpy(), xn, "f32", chat, ref, gap)
