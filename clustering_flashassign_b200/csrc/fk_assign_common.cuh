@@ -1,8 +1,7 @@
-// Device helpers shared by the two FlashAssign kernels (one CTA per point
-// tile in fk_assign_tc.cu, a CTA pair per 256-point tile in fk_assign_pair.cu):
-// the packed-key and exact running argmax over TMEM loads, the point-norm sums
-// of a shared tile, the 32-byte-swizzled norm-row stores, and the exact fp64
-// re-rank of points far from every centroid.
+// Device helpers of the FlashAssign kernels: the packed-key and exact running
+// argmax over TMEM loads, the point-norm sums of a shared tile, the
+// 32-byte-swizzled norm-row stores, and the exact fp64 re-rank of points far
+// from every centroid.
 #pragma once
 
 #include <cuda.h>

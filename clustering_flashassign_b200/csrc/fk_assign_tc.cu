@@ -9,10 +9,11 @@
 // exists": point tiles and centroid chunks are streamed on chip and the cross
 // term never leaves it).
 //
-// Mapping on a B200 SM (one persistent CTA per SM, 352 threads):
-//   warp 0      TMA producer: point tiles (128 x d), centroid chunks (256 x 64
-//               K-blocks) into 128-byte-swizzled shared memory, and each
-//               chunk's norm rows (256 x 16, 32-byte swizzle),
+// Mapping on a B200 SM (one persistent CTA per SM, 384 threads):
+//   warp 0      TMA producer: centroid chunks (256 x 64 K-blocks) into
+//               128-byte-swizzled shared memory and each chunk's norm rows
+//               (256 x 16, 32-byte swizzle); split-d: the point tile's
+//               K-blocks too,
 //   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16, kind::f16)
 //               into a TMEM accumulator; two accumulators (2 x 256 columns =
 //               all 512 TMEM columns) let the MMA of chunk c+1 overlap the
@@ -25,7 +26,14 @@
 //               and split the chunk's columns; their results are combined
 //               once per point tile,
 //   warp 10     (resident variant) ||x||^2 of each point tile from the shared
-//               copy, written as the tile's norm rows.
+//               copy, written as the tile's norm rows,
+//   warp 11     (resident variant) the point tiles (128 x d), one tile ahead.
+// The MMA thread is the pipeline's serial point, so in the resident variant
+// it waits on one barrier per chunk and commits once: the producer, after
+// issuing a chunk's copies, also waits for the chunk's accumulator to be free
+// (and, for a tile's first chunk, for the tile's norm rows) and then arrives
+// on the stage's full barrier a second time; the chunk's single commit frees
+// the stage and tells the epilogue that the accumulator is complete.
 // Two variants, picked by d:
 //   resident X (d <= 128): the point tile stays in shared memory for all K
 //               chunks (double-buffered across tiles); only centroids stream.
@@ -56,6 +64,10 @@
 //               item, consecutive CTAs taking one tile's chunks so they share
 //               its reads in L2; the chunks merge by a 64-bit atomicMax per
 //               point and k_keys_to_ids writes the ids.
+// Every role waits by polling its mbarriers without suspending (a suspended
+// thread resumes hundreds of cycles after the phase completes, and the
+// per-chunk hand-offs between the roles are on the tensor core's critical
+// path); each wait still gives up after the time limit or on the CTA's abort.
 // Rows past N and centroid rows past K are zero-filled by TMA; padded centroid
 // columns carry a sentinel norm row (acc about -2^31 or below) so they never win.
 #include <cuda.h>
@@ -69,7 +81,8 @@ using namespace sm100;
 
 constexpr int kEpiWarps = 8;
 constexpr int kNormWarp = 2 + kEpiWarps;
-constexpr int kThreads = 32 * (kNormWarp + 1);
+constexpr int kLoadWarp = kNormWarp + 1;  // resident: point-tile copies
+constexpr int kThreads = 32 * (kLoadWarp + 1);
 constexpr uint32_t kXBlockBytes = kTileM * kBlockK * 2;   // 16 KB
 constexpr uint32_t kCBlockBytes = kChunkN * kBlockK * 2;  // 32 KB
 constexpr uint32_t kAExtBytes = kTileM * kExt * 2;        // 4 KB of point norm rows
@@ -132,7 +145,7 @@ struct Layout {
   static constexpr uint32_t kMergeOff = (kMiscOff + 16 + 15) / 16 * 16;
   // resident: ||x||^2 of the rows of the two point-tile buffers, for the
   // epilogue's far-point check
-  static constexpr uint32_t kXnOff = kMergeOff + 2 * kTileM * 8;
+  static constexpr uint32_t kXnOff = kMergeOff + kTileM * 16;
   static constexpr uint32_t kBytes = kXnOff + (RESIDENT ? 2 * kTileM * 4 : 0);
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
   static_assert(kStagesOff % 1024 == 0, "swizzled tiles need 1024-byte alignment");
@@ -155,7 +168,7 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, int *e
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                           int *err, int lane) {
   int r = 1;
-  if (lane == 0) r = mbar_wait(bar, parity, abort_flag, err) ? 1 : 0;
+  if (lane == 0) r = mbar_wait_spin(bar, parity, abort_flag, err) ? 1 : 0;
   r = __shfl_sync(0xffffffffu, r, 0);
   __syncwarp();
   return r != 0;
@@ -193,13 +206,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *xnorm_s = reinterpret_cast<float *>(smem + L::kXnOff);  // [2][kTileM], resident only
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
-  float2 *merge = reinterpret_cast<float2 *>(smem + L::kMergeOff);
+  float4 *merge = reinterpret_cast<float4 *>(smem + L::kMergeOff);  // [kTileM]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full(s), 1);
+      // resident: the producer arrives twice, once with the copies' byte count
+      // and once when the chunk's accumulator (and, for a tile's first chunk,
+      // the tile's norm rows) are free to use
+      mbar_init(full(s), RESIDENT ? 2 : 1);
       mbar_init(empty(s), 1);
     }
     for (int e = 0; e < kExtSlots; ++e) {
@@ -263,57 +279,50 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t f = 0, g = 0, e = 0;
+      uint32_t f = 0, e = 0, u = 0;  // stages, ext rows, tiles done
       bool ok = true;
-      // Point tiles are loaded one tile ahead: the tile after this one is
-      // requested right after this tile's first chunk, as soon as the MMAs of
-      // the tile before have released its buffer, so the norm warp has a whole
-      // tile of time for it.
-      auto load_x = [&](int tile) -> bool {
-        const int xb = g & 1;
-        if (!mbar_wait(xempty(xb), ((g >> 1) & 1) ^ 1, abort_flag, a.err)) return false;
-        mbar_arrive_expect_tx(xfull(xb), KB * kXBlockBytes);
-        const int b = tile / a.tiles_per_batch;
-        const int row0 = (tile % a.tiles_per_batch) * kTileM;
-        for (int kb = 0; kb < KB; ++kb)
-          tma_load_3d(&tmx, x_base + (xb * KB + kb) * kXBlockBytes, xfull(xb), kb * kBlockE, row0, b);
-        ++g;
-        return true;
-      };
-      if (RESIDENT && (int)blockIdx.x < a.total_tiles) ok = load_x(blockIdx.x);
       for (int task = blockIdx.x; ok && task < ntask; task += gridDim.x) {
         const int tile = task_tile(task);
         const int b = tile / a.tiles_per_batch;
         const int row0 = (tile % a.tiles_per_batch) * kTileM;
         for (int c = chunk_lo(task); ok && c < chunk_hi(task); ++c) {
           if (RESIDENT) {  // the whole chunk and its norm rows in one stage
+            // empty(s) is committed once per chunk by the MMA thread: the
+            // stage is free and the epilogue may read the chunk's accumulator
             const int s = f % STAGES;
-            if (!mbar_wait(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+            if (!mbar_wait_spin(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
             const uint32_t dst = st_base + s * L::kStageBytes;
             mbar_arrive_expect_tx(full(s), L::kStageBytes);
             for (int kb = 0; kb < KB; ++kb)
               tma_load_3d(&tmc, dst + kb * kCBlockBytes, full(s), kb * kBlockE, c * kChunkN, b);
             tma_load_3d(&tme, dst + KB * kCBlockBytes, full(s), 0, c * kChunkN, b);
+            // The MMA thread waits on full(s) alone: this thread takes the
+            // other waits of the chunk off its path between two chunks.
+            bool ready = true;
+            if (c == 0)  // the tile's point norm rows are written (so its copy landed too)
+              ready = mbar_wait_spin(xnfull(u & 1), (u >> 1) & 1, abort_flag, a.err);
+            ready = ready && mbar_wait_spin(accempty(f & 1), ((f >> 1) & 1) ^ 1, abort_flag, a.err);
+            mbar_arrive(full(s));  // also when aborting, so the phase completes as the copies land
             ++f;
+            if (!ready) { ok = false; break; }
           } else {  // this chunk's centroid norm rows (used by the chunk's last MMA step)
             const int es = e % kExtSlots;
-            if (!mbar_wait(eempty(es), ((e / kExtSlots) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+            if (!mbar_wait_spin(eempty(es), ((e / kExtSlots) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
             mbar_arrive_expect_tx(efull(es), kBExtBytes);
             tma_load_3d(&tme, bext_base + es * kBExtBytes, efull(es), 0, c * kChunkN, b);
             ++e;
           }
           for (int kb = 0; !RESIDENT && kb < kblocks; ++kb) {
             const int s = f % STAGES;
-            if (!mbar_wait(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+            if (!mbar_wait_spin(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
             const uint32_t dst = st_base + s * L::kStageBytes;
             mbar_arrive_expect_tx(full(s), kXBlockBytes + kCBlockBytes);
             tma_load_3d(&tmx, dst, full(s), kb * kBlockE, row0, b);
             tma_load_3d(&tmc, dst + kXBlockBytes, full(s), kb * kBlockE, c * kChunkN, b);
             ++f;
           }
-          if (RESIDENT && ok && c == 0 && tile + (int)gridDim.x < a.total_tiles)
-            ok = load_x(tile + gridDim.x);
         }
+        ++u;
       }
       // tail: make every issued copy and every release of a buffer land before exit
       const bool aborted = *abort_flag != 0;
@@ -321,10 +330,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         wait_drain(aborted ? full(ff % STAGES) : empty(ff % STAGES), (ff / STAGES) & 1, a.err);
       for (uint32_t ee = e > (uint32_t)kExtSlots ? e - kExtSlots : 0; ee < e; ++ee)
         wait_drain(aborted ? efull(ee % kExtSlots) : eempty(ee % kExtSlots), (ee / kExtSlots) & 1, a.err);
-      if (RESIDENT) {
-        for (uint32_t gg = g > 2 ? g - 2 : 0; gg < g; ++gg)
-          wait_drain(aborted ? xfull(gg & 1) : xempty(gg & 1), (gg >> 1) & 1, a.err);
-      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -336,21 +341,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         int xb = 0;
         if (RESIDENT) {
           xb = g & 1;
-          if (!mbar_wait(xfull(xb), (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+          if (!mbar_wait_spin(xfull(xb), (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
         }
         const uint32_t a_ext = aext_base + (RESIDENT ? xb * kAExtBytes : 0u);
         for (int c = chunk_lo(task); ok && c < chunk_hi(task); ++c) {
           const int ab = h & 1;
-          if (!mbar_wait(accempty(ab), ((h >> 1) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem + ab * kChunkN;
           if (RESIDENT) {
-            if (c == 0) {  // the tile's point norm rows are written
-              if (!mbar_wait(xnfull(xb), (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
-            }
+            // full(s) also stands for the free accumulator and the tile's norm
+            // rows (the producer's second arrival); one commit per chunk to
+            // empty(s) frees the stage and hands the accumulator to the epilogue
+            const uint32_t d_tmem = tmem + ab * kChunkN;
             const int s = f % STAGES;
-            if (!mbar_wait(full(s), (f / STAGES) & 1, abort_flag, a.err)) { ok = false; break; }
+            if (!mbar_wait_spin(full(s), (f / STAGES) & 1, abort_flag, a.err)) { ok = false; break; }
             tc_fence_after();
             const uint32_t stage = st_base + s * L::kStageBytes;
 #pragma unroll
@@ -364,15 +367,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // the norm step: acc += A_ext . B_ext (fk_norms.cuh)
             mma_t<T>(d_tmem, desc_k_sw32(a_ext), desc_k_sw32(stage + KB * kCBlockBytes), a.idesc, 1u);
-            mma_commit(empty(s));  // frees the stage once these MMAs have read it
+            mma_commit(empty(s));  // stage free, accumulator complete
             ++f;
-            mma_commit(accfull(ab));  // accumulator ready for the epilogue
             ++h;
             continue;
           }
+          if (!mbar_wait_spin(accempty(ab), ((h >> 1) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + ab * kChunkN;
           for (int kb = 0; kb < kblocks; ++kb) {
             const int s = f % STAGES;
-            if (!mbar_wait(full(s), (f / STAGES) & 1, abort_flag, a.err)) { ok = false; break; }
+            if (!mbar_wait_spin(full(s), (f / STAGES) & 1, abort_flag, a.err)) { ok = false; break; }
             tc_fence_after();
             const uint32_t stage = st_base + s * L::kStageBytes;
             const uint32_t a_addr = RESIDENT ? x_base + (xb * KB + kb) * kXBlockBytes : stage;
@@ -387,11 +392,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           // the norm step: acc += A_ext . B_ext (fk_norms.cuh)
           if (RESIDENT && c == 0) {
-            if (!mbar_wait(xnfull(xb), (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+            if (!mbar_wait_spin(xnfull(xb), (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
             tc_fence_after();
           }
           const int es = e % kExtSlots;
-          if (!mbar_wait(efull(es), (e / kExtSlots) & 1, abort_flag, a.err)) { ok = false; break; }
+          if (!mbar_wait_spin(efull(es), (e / kExtSlots) & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
           mma_t<T>(d_tmem, desc_k_sw32(a_ext), desc_k_sw32(bext_base + es * kBExtBytes), a.idesc, 1u);
           mma_commit(eempty(es));
@@ -411,8 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kNormWarp) {
     // ------------------------------------------------------------ point norms
     if constexpr (RESIDENT) {
+      bool ok = true;
       uint32_t g = 0;
-      for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++g) {
+      for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x, ++g) {
         const int xb = g & 1;
         const int b = tile / a.tiles_per_batch;
         const int row0 = (tile % a.tiles_per_batch) * kTileM;
@@ -473,6 +479,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(xnfull(xb));
       }
     }
+  } else if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ point tiles
+    // (resident) tile g goes into the buffer of tile g - 2 as soon as that
+    // tile's MMAs are done, so it is requested a whole tile ahead of its use
+    if (RESIDENT && lane == 0) {
+      uint32_t g = 0;
+      for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++g) {
+        const int xb = g & 1;
+        if (!mbar_wait_spin(xempty(xb), ((g >> 1) & 1) ^ 1, abort_flag, a.err)) break;
+        mbar_arrive_expect_tx(xfull(xb), KB * kXBlockBytes);
+        const int b = tile / a.tiles_per_batch;
+        const int row0 = (tile % a.tiles_per_batch) * kTileM;
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_3d(&tmx, x_base + (xb * KB + kb) * kXBlockBytes, xfull(xb), kb * kBlockE, row0, b);
+      }
+      // tail: the issued copies land (or are consumed) before exit
+      const bool aborted = *abort_flag != 0;
+      for (uint32_t gg = g > 2 ? g - 2 : 0; gg < g; ++gg)
+        wait_drain(aborted ? xfull(gg & 1) : xempty(gg & 1), (gg >> 1) & 1, a.err);
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
@@ -491,9 +518,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = (tile % a.tiles_per_batch) * kTileM;
       float best = __int_as_float(0xff800000);  // -inf
       int bidx = 0;                              // chunk (packed) or column (exact) of best
+      float xn = 0.f;                            // ||x||^2 of this row (resident, half 1)
       for (int c = chunk_lo(task); c < chunk_hi(task); ++c, ++h) {
         const int ab = h & 1;
-        if (!warp_wait(accfull(ab), (h >> 1) & 1, abort_flag, a.err, lane)) { ok = false; break; }
+        // resident: the chunk's one commit (empty of its stage) marks the
+        // accumulator complete; the barrier cannot run a phase ahead, since the
+        // chunk STAGES later needs this warp's release of a later chunk first
+        const bool got = RESIDENT ? warp_wait(empty(h % STAGES), (h / STAGES) & 1, abort_flag, a.err, lane)
+                                  : warp_wait(accfull(ab), (h >> 1) & 1, abort_flag, a.err, lane);
+        if (!got) { ok = false; break; }
         tc_fence_after();
         const uint32_t tb = t_lane + ab * kChunkN;
         uint32_t ra[32], rb[32], rc[32], rd[32];
@@ -510,6 +543,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(accempty(ab));  // accumulator may be overwritten
+          if (half == 1 && c == chunk_lo(task)) {
+            // ||x||^2 for the far-point check (header), read once per tile by
+            // the warps that do not write the ids, off the tile's critical
+            // end; xnfull completed before this tile's first MMA, and waiting
+            // on it orders the norm warp's stores before these reads
+            if (!warp_wait(xnfull(u & 1), (u >> 1) & 1, abort_flag, a.err, lane)) { ok = false; break; }
+            xn = xnorm_s[(u & 1) * kTileM + r_in_tile];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xnfree(u & 1));  // the norm warp may reuse the slot
+          }
           scan_packed(rc, 64, colb, m0, m1, m2, m3);
           scan_packed(rd, 96, colb, m0, m1, m2, m3);
           const float m = fmaxf(max3f(m0, m1, m2), m3);
@@ -555,20 +598,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         val = best;
         idx = bidx;
       }
-      // combine the two column halves of each row: larger value, then lower index
-      const int p = u & 1;
-      const uint32_t vpar = (u >> 1) & 1;
-      float2 *slot = merge + p * kTileM + r_in_tile;
+      // combine the two column halves of each row: larger value, then lower
+      // index (one slot per row: the half-1 warps write a tile's slot a whole
+      // tile after the half-0 warps read the previous one)
+      const uint32_t vpar = u & 1;
+      float4 *slot = merge + r_in_tile;
       if (half == 1) {
-        if (!warp_wait(mempty(p), vpar ^ 1, abort_flag, a.err, lane)) { ok = false; break; }
-        *slot = make_float2(val, __int_as_float(idx));
+        if (!warp_wait(mempty(0), vpar ^ 1, abort_flag, a.err, lane)) { ok = false; break; }
+        *slot = make_float4(val, __int_as_float(idx), xn, 0.f);
         __syncwarp();
-        if (lane == 0) mbar_arrive(mfull(p));
+        if (lane == 0) mbar_arrive(mfull(0));
       } else {
-        if (!warp_wait(mfull(p), vpar, abort_flag, a.err, lane)) { ok = false; break; }
-        const float2 o = *slot;
+        if (!warp_wait(mfull(0), vpar, abort_flag, a.err, lane)) { ok = false; break; }
+        const float4 o = *slot;
         __syncwarp();
-        if (lane == 0) mbar_arrive(mempty(p));
+        if (lane == 0) mbar_arrive(mempty(0));
         const float ov = o.x;
         const int oi = __float_as_int(o.y);
         if (ov > val || (ov == val && oi < idx)) {  // the value travels too: the keys compare it
@@ -579,13 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (RESIDENT) {
           // far-point check (see the header): flagged rows of this warp are
           // re-ranked one after another by the whole warp
-          // xnfull of this tile completed before its first MMA; waiting on it
-          // here orders the norm warp's stores before these reads
-          if (!warp_wait(xnfull(p), (u >> 1) & 1, abort_flag, a.err, lane)) { ok = false; break; }
-          const float xn = xnorm_s[p * kTileM + r_in_tile];
-          __syncwarp();
-          if (lane == 0) mbar_arrive(xnfree(p));  // the norm warp may reuse the slot
-          unsigned flagged = __ballot_sync(0xffffffffu, row < a.N && -val > kFarRatioHalf * xn);
+          unsigned flagged = __ballot_sync(0xffffffffu, row < a.N && -val > kFarRatioHalf * o.z);
           while (flagged) {
             const int src = __ffs(flagged) - 1;
             flagged &= flagged - 1;

@@ -21,3 +21,4 @@ def _gpu_guard(request):
         if not torch.cuda.is_available():
             pytest.fail("GPU test run without a visible CUDA device")
     yield
+

@@ -46,6 +46,8 @@ ASSIGN_CASES = [
     (2, 300, 257, 128, "f16"),     # one centroid past a chunk
     (1, 64, 1, 16, "f16"),         # K = 1, N below one tile
     (1, 256, 256, 32, "f16"),      # K = N
+    (3, 40000, 700, 128, "f16"),   # 939 point tiles: several tiles per CTA
+    (2, 45000, 520, 64, "bf16"),   # the same with one K-block, ragged last tile of each batch
 ]
 
 
