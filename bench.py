@@ -68,7 +68,7 @@ def kernel_source_hash():
     internal header, so host-side declarations there do not count as a change."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "clustering_flashassign_b200", "csrc")
-    for name in ["fk_assign_tc.cu", "fk_sm100.cuh", "fk_norms.cuh"]:
+    for name in ["fk_assign_tc.cu", "fk_assign_common.cuh", "fk_sm100.cuh", "fk_norms.cuh"]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     with open(os.path.join(csrc, "fk_internal.h")) as f:
@@ -548,6 +548,16 @@ def run_largen(args):
     fk.fk_profile_enable(False)
     prof = fk.fk_profile_read(reset=True)
     ms = e0.elapsed_time(e1)
+    # one more iteration with the per-chunk timeline (outside the timed region):
+    # each chunk's copy must end before its compute begins (the stream waits
+    # on it), and the copy of chunk j + 1 should run while chunk j computes
+    fk.fk_profile_enable(3)
+    fk.fk_lloyd(xt, initd, 1, 0.0, ids, cen, host_mode=fk.FK_HOST_STREAM)
+    torch.cuda.synchronize()
+    fk.fk_profile_enable(False)
+    fk.fk_profile_read(reset=True)
+    tl = fk.fk_profile_timeline()
+    timeline = timeline_summary(tl)
     peaks, src_name = load_peaks()
     peak_t = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
     flop_iter = 2.0 * w.B * w.N * w.K * w.d
@@ -581,8 +591,34 @@ def run_largen(args):
                          "sample": f"one iteration on the first {ns} points with all K, extrapolated x{w.N // ns}"},
         "gpu_launches": fk.fk_launch_count() - launches0,
         "clocks": clk.summary(),
+        "timeline": timeline,
     }
     print(json.dumps(line), flush=True)
+
+
+def timeline_summary(tl):
+    """Per-chunk copy / compute events of one streamed iteration, summarised:
+    how long copies and computes take, whether every copy ended before its
+    compute began, and how much of each copy ran under the previous chunk's
+    compute."""
+    if not tl:
+        return None
+    copy = [c["copy_end"] - c["copy_begin"] for c in tl]
+    comp = [c["compute_end"] - c["compute_begin"] for c in tl]
+    before = sum(1 for c in tl if c["copy_end"] <= c["compute_begin"] + 1e-6)
+    hidden = []
+    for prev, cur in zip(tl, tl[1:]):
+        # the part of this chunk's copy that ran while the previous chunk computed
+        lo, hi = max(cur["copy_begin"], prev["compute_begin"]), min(cur["copy_end"], prev["compute_end"])
+        span = cur["copy_end"] - cur["copy_begin"]
+        hidden.append(max(0.0, hi - lo) / span if span > 0 else 1.0)
+    gaps = [cur["compute_begin"] - prev["compute_end"] for prev, cur in zip(tl, tl[1:])]
+    return {"chunks": len(tl), "copy_ms_mean": statistics.mean(copy), "compute_ms_mean": statistics.mean(comp),
+            "copies_ended_before_their_compute": before,
+            "copy_hidden_under_previous_compute_mean": statistics.mean(hidden) if hidden else None,
+            "compute_gap_ms_max": max(gaps) if gaps else 0.0,
+            "span_ms": tl[-1]["compute_end"] - tl[0]["copy_begin"],
+            "first_chunks": [{k: round(v, 3) if isinstance(v, float) else v for k, v in c.items()} for c in tl[:4]]}
 
 
 def baseline_assign_materialised(xd, cd):

@@ -38,7 +38,7 @@ FK_FAULT_NONE, FK_FAULT_ALLOC, FK_FAULT_H2D, FK_FAULT_LAUNCH = 0, 1, 2, 3
 DTYPES = {torch.float32: FK_F32, torch.float16: FK_F16, torch.bfloat16: FK_BF16}
 
 EXPORTS = ["fk_assign", "fk_update", "fk_sort", "fk_lloyd", "fk_assign_noalloc", "fk_status_string",
-           "fk_last_error", "fk_device_error", "fk_release", "fk_profile_enable", "fk_profile_read",
+           "fk_last_error", "fk_device_error", "fk_release", "fk_profile_enable", "fk_profile_read", "fk_profile_timeline",
            "fk_launch_count", "fk_version", "fk_selftest_bounded_wait", "fk_point_norms",
            "fk_init_centers", "fk_lloyd_step_partial", "fk_update_finalize", "fk_inject_fault"]
 
@@ -84,6 +84,7 @@ def _load():
         "fk_release": (I, []),
         "fk_profile_enable": (I, [I]),
         "fk_profile_read": (I, [ctypes.POINTER(FkProfile), I]),
+        "fk_profile_timeline": (I, [P, I, ctypes.POINTER(I)]),
         "fk_launch_count": (LL, []),
         "fk_version": (I, []),
         "fk_selftest_bounded_wait": (I, [LL, P]),
@@ -275,7 +276,8 @@ def fk_release() -> None:
 
 
 def fk_profile_enable(on=True) -> None:
-    """0 / False: off; 1 / True: every phase; 2: assign and whole update only."""
+    """0 / False: off; 1 / True: every phase; 2: assign and whole update only;
+    3: as 2, plus the streamed pipeline's per-chunk timeline (fk_profile_timeline)."""
     _check(lib.fk_profile_enable(int(on)), "fk_profile_enable")
 
 
@@ -283,6 +285,19 @@ def fk_profile_read(reset: bool = False) -> dict:
     p = FkProfile()
     _check(lib.fk_profile_read(ctypes.byref(p), 1 if reset else 0), "fk_profile_read")
     return {f: getattr(p, f) for f, _ in FkProfile._fields_}
+
+
+def fk_profile_timeline(max_chunks: int = 4096):
+    """Per-chunk events of the streamed pipeline recorded at profile level 3:
+    a list of dicts {chunk, buf, copy_begin, copy_end, compute_begin,
+    compute_end} in ms from the first copy (clears the record)."""
+    import numpy as np
+    out = np.zeros((max_chunks, 6), np.float64)
+    n = ctypes.c_int(0)
+    _check(lib.fk_profile_timeline(ctypes.c_void_p(out.ctypes.data), max_chunks, ctypes.byref(n)),
+           "fk_profile_timeline")
+    keys = ("chunk", "buf", "copy_begin", "copy_end", "compute_begin", "compute_end")
+    return [dict(zip(keys, (int(r[0]), int(r[1]), *map(float, r[2:])))) for r in out[: n.value]]
 
 
 def fk_launch_count() -> int:

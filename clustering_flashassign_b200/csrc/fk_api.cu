@@ -243,10 +243,13 @@ int streamed_pass(Workspace *ws, const fk_shape &sh, const char *xh, long long c
       void *xb = ws->chunk[buf].p;
       FK_CUDA(cudaStreamWaitEvent(ws->copy_stream, ws->freed[buf], 0));
       if (fault_hit(FK_FAULT_H2D)) return set_error(FK_ECUDA, "injected host-to-device copy failure (FK_FAULT)");
+      FK_TRY(chunk_event(0, ws->stream_job, buf, ws->copy_stream));
       FK_CUDA(cudaMemcpyAsync(xb, xh + ((size_t)b * N + n0) * d * es, (size_t)nc * d * es,
                               cudaMemcpyHostToDevice, ws->copy_stream));
+      FK_TRY(chunk_event(1, ws->stream_job, buf, ws->copy_stream));
       FK_CUDA(cudaEventRecord(ws->ready[buf], ws->copy_stream));
       FK_CUDA(cudaStreamWaitEvent(s, ws->ready[buf], 0));
+      FK_TRY(chunk_event(2, ws->stream_job, buf, s));
       int32_t *idc = ids_dev + (size_t)b * N + n0;
       const void *cb = (const char *)cassign + (size_t)b * K * d * es;
       FK_TRY(do_assign_resident(ws, xb, cb, cnx ? cnx + ext_bytes(b, Kpad) : nullptr, nullptr, 1, nc, K,
@@ -261,6 +264,7 @@ int streamed_pass(Workspace *ws, const fk_shape &sh, const char *xh, long long c
         FK_TRY(launch_accumulate(sums, first, pieces_of(nc), counts, offsets, 1, K, d,
                                  gsum + (size_t)b * K * d, gcounts + (size_t)b * K, false, s));
       }
+      FK_TRY(chunk_event(3, ws->stream_job, buf, s));
       FK_CUDA(cudaEventRecord(ws->freed[buf], s));
     }
   }
@@ -703,6 +707,14 @@ int fk_release(void) {
 int fk_profile_enable(int on) { return profile_enable(on); }
 
 int fk_profile_read(fk_profile *out, int reset) { return profile_read(out, reset); }
+
+int fk_profile_timeline(double *out, int max_chunks, int *rows) {
+  if (max_chunks < 0) return set_error(FK_EINVAL, "max_chunks must be >= 0");
+  int n = 0;
+  FK_TRY(profile_timeline(out, max_chunks, &n));
+  if (rows) *rows = n;
+  return FK_OK;
+}
 
 long long fk_launch_count(void) { return launch_count(); }
 

@@ -104,6 +104,12 @@ int release_device_workspaces();
 long long launch_count();
 int profile_enable(int on);
 int profile_read(fk_profile *out, int reset);
+// Level 3: per-chunk events of the streamed pipeline.  which: 0 copy begin,
+// 1 copy end (on the copy stream), 2 compute begin, 3 compute end (on the
+// compute stream); 0 opens the chunk's record.
+bool timeline_on();
+int chunk_event(int which, long long chunk, int buf, cudaStream_t s);
+int profile_timeline(double *out, int max_chunks, int *rows);
 const char *last_error();
 
 size_t esize(int dtype);

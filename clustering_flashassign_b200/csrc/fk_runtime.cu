@@ -28,6 +28,14 @@ struct Pending {
 std::vector<Pending> g_pending;
 double g_ms[PH_COUNT] = {0, 0, 0, 0, 0};
 long long g_assign_launches = 0, g_update_calls = 0, g_prof_launches = 0;
+// level 3: per-chunk events of the streamed pipeline (copy begin / end on the
+// copy stream, compute begin / end on the compute stream)
+struct ChunkEvents {
+  cudaEvent_t ev[4];
+  long long chunk;
+  int buf;
+};
+std::vector<ChunkEvents> g_chunks;
 }  // namespace
 
 int set_error(int status, const std::string &msg) {
@@ -227,7 +235,7 @@ cudaEvent_t take_event() {
 
 PhaseTimer::PhaseTimer(int ph, cudaStream_t st) : phase(ph), s(st) {
   if (!g_prof_level) return;
-  if (g_prof_level == 2 && ph != PH_ASSIGN && ph != PH_UPDATE) return;
+  if (g_prof_level >= 2 && ph != PH_ASSIGN && ph != PH_UPDATE) return;
   a = take_event();
   b = take_event();
   if (!a || !b) {
@@ -252,8 +260,51 @@ void note_update_call() {
 }
 
 int profile_enable(int on) {
-  if (on < 0 || on > 2) return set_error(FK_EINVAL, "profile level must be 0, 1 or 2");
+  if (on < 0 || on > 3) return set_error(FK_EINVAL, "profile level must be 0, 1, 2 or 3");
   g_prof_level = on;
+  return FK_OK;
+}
+
+bool timeline_on() { return g_prof_level == 3; }
+
+int chunk_event(int which, long long chunk, int buf, cudaStream_t s) {
+  if (g_prof_level != 3) return FK_OK;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (which == 0) {
+    ChunkEvents c;
+    c.chunk = chunk;
+    c.buf = buf;
+    for (auto &e : c.ev) FK_CUDA(cudaEventCreate(&e));
+    g_chunks.push_back(c);
+  }
+  if (g_chunks.empty() || g_chunks.back().chunk != chunk) return set_error(FK_EINVAL, "chunk events out of order");
+  FK_CUDA(cudaEventRecord(g_chunks.back().ev[which], s));
+  return FK_OK;
+}
+
+int profile_timeline(double *out, int max_chunks, int *rows) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  int n = 0;
+  float t0 = 0.f;
+  for (size_t i = 0; i < g_chunks.size(); ++i) {
+    auto &c = g_chunks[i];
+    FK_CUDA(cudaEventSynchronize(c.ev[3]));
+    if (out && n < max_chunks) {
+      double *row = out + 6 * (size_t)n;
+      row[0] = (double)c.chunk;
+      row[1] = (double)c.buf;
+      for (int k = 0; k < 4; ++k) {
+        float ms = 0.f;
+        FK_CUDA(cudaEventElapsedTime(&ms, g_chunks[0].ev[0], c.ev[k]));
+        row[2 + k] = ms - t0;
+      }
+      ++n;
+    }
+  }
+  for (auto &c : g_chunks)
+    for (auto &e : c.ev) cudaEventDestroy(e);
+  g_chunks.clear();
+  *rows = n;
   return FK_OK;
 }
 

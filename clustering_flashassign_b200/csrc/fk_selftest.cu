@@ -1,7 +1,8 @@
 // fk_selftest_bounded_wait: exercises the bounded-wait path every tcgen05
 // kernel of the library relies on, without any fault.  One CTA initialises an
 // mbarrier that nothing ever arrives at and waits on it with the library's
-// wait loop (try_wait with a suspend hint, %globaltimer limit).  When the
+// wait loop (the FlashAssign roles poll with mbarrier.test_wait and check the
+// %globaltimer limit every 256 polls).  When the
 // limit expires the kernel records DEV_TIMEOUT in the stream's device error
 // word and returns; the host reads it as FK_ETIMEOUT and the context stays
 // usable.
@@ -21,10 +22,11 @@ __global__ void k_wait_selftest(unsigned long long limit_ns, int *err) {
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    // the same loop as mbar_wait, with the caller's limit instead of 2 s
+    // the same loop as mbar_wait_spin, with the caller's limit instead of 2 s
     const uint64_t t0 = sm100::globaltimer();
-    for (;;) {
-      if (sm100::mbar_try_wait_sleep(b, 0, 200000u)) break;  // never: nothing arrives
+    for (uint32_t n = 1;; ++n) {
+      if (sm100::mbar_test(b, 0)) break;  // never: nothing arrives
+      if ((n & 255u) != 0) continue;
       if (abort_flag) break;
       if (sm100::globaltimer() - t0 > limit_ns) {
         abort_flag = 1;

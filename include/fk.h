@@ -351,8 +351,23 @@ typedef struct {
 
 /* Event timing: 0 off (default), 1 every phase (assign, sort, reduce,
  * finalize, whole update), 2 light (assign and whole update only: two event
- * pairs per Lloyd iteration). */
+ * pairs per Lloyd iteration), 3 as 2 plus a timeline of the streamed
+ * pipeline's chunks (fk_profile_timeline). */
 int fk_profile_enable(int on);
+
+/*
+ * fk_profile_timeline -- the chunks streamed while the level was 3, in issue
+ * order: six doubles per chunk, {chunk number, device buffer (0 or 1),
+ * copy begin, copy end (on the copy stream), compute begin, compute end (on
+ * the compute stream: assign, sort and segment reduce of the chunk)}, times
+ * in ms from the first chunk's copy begin.  Writes at most max_chunks rows to
+ * out (host; NULL discards them) and their number to *rows (host, nullable),
+ * synchronizes the recorded events and clears the record.  FK_EINVAL for
+ * max_chunks < 0.  It measures the chunked host-to-device overlap
+ * ("Flash-KMeans: Fast and Memory-Efficient Exact K-Means", Abstract:
+ * chunked-stream overlap); an interface addition, the pages show no timeline.
+ */
+int fk_profile_timeline(double *out, int max_chunks, int *rows);
 
 /* Synchronizes the recorded events, fills *out, and clears the totals if reset != 0. */
 int fk_profile_read(fk_profile *out, int reset);

@@ -90,3 +90,34 @@ def test_largen_streamed_matches_device_resident_run():
     assert torch.equal(out[0][0], out[1][0])
     # sums are folded chunk by chunk in the streamed run: equal up to fp32 rounding
     torch.testing.assert_close(out[0][1], out[1][1], rtol=1e-5, atol=1e-5)
+
+
+def test_streamed_timeline_shows_copies_before_their_compute_and_overlap():
+    """Profile level 3 records, per streamed chunk, the copy (copy stream) and
+    the compute (compute stream): each copy ends before its chunk's compute
+    begins, and the copy of chunk j + 1 starts before chunk j's compute ends
+    (the double buffer overlaps them)."""
+    import clustering_flashassign_b200 as fk
+    w = synthdata.scaled(synthdata.WORKLOADS["largen"], N=1 << 21, K=4096)
+    xt = torch.empty((w.B, w.N, w.d), dtype=torch.float16, pin_memory=True)
+    _, _, init = synthdata.make(w, out=xt.numpy())
+    initd = torch.from_numpy(init).cuda()
+    ids = torch.empty((w.B, w.N), dtype=torch.int32, device="cuda")
+    cen = torch.empty((w.B, w.K, w.d), dtype=torch.float32, device="cuda")
+    fk.fk_lloyd(xt, initd, 1, 0.0, ids, cen, host_mode=fk.FK_HOST_STREAM, chunk_points=1 << 18)  # warm-up
+    fk.fk_profile_timeline()  # nothing recorded at level 0
+    fk.fk_profile_enable(3)
+    try:
+        fk.fk_lloyd(xt, initd, 2, 0.0, ids, cen, host_mode=fk.FK_HOST_STREAM, chunk_points=1 << 18)
+        torch.cuda.synchronize()
+    finally:
+        fk.fk_profile_enable(False)
+        fk.fk_profile_read(reset=True)
+    tl = fk.fk_profile_timeline()
+    assert len(tl) == 2 * 8
+    assert [c["buf"] for c in tl] == [c["chunk"] & 1 for c in tl]
+    for c in tl:
+        assert c["copy_begin"] <= c["copy_end"] <= c["compute_begin"] + 1e-3 <= c["compute_end"] + 1e-3
+    overlapped = sum(1 for a, b in zip(tl, tl[1:]) if b["copy_begin"] < a["compute_end"])
+    assert overlapped >= len(tl) // 2
+    assert fk.fk_profile_timeline() == []  # read once, then cleared
