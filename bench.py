@@ -437,6 +437,10 @@ def run_fk(args, rank, world, local_rank, dist):
     cpu_t1 = cpu_oracle_sample(x, init, w, 1, threads=1, points=pts1)
     cpu_value_1t = 1.0 / (cpu_t1 * w.B * (w.N / pts1))
 
+    others = None
+    if w.name == WORKLOAD and not args.no_workloads:
+        others = {name: time_workload(name, dev) for name in OTHER_WORKLOADS}
+
     baselines = None
     if w.name == WORKLOAD and not args.no_baselines:
         # the pages' two comparison kernels (materialised distances, scatter
@@ -489,6 +493,8 @@ def run_fk(args, rank, world, local_rank, dist):
     }
     if baselines is not None:
         line["baselines"] = baselines
+    if others is not None:
+        line["workloads"] = others
     print(json.dumps(line), flush=True)
 
 
@@ -594,6 +600,50 @@ def run_largen(args):
         "timeline": timeline,
     }
     print(json.dumps(line), flush=True)
+
+
+# The other workloads of the parity suite, each timed briefly after the main
+# measurement (not part of its timed region): CUDA events around fk_lloyd calls
+# on device-resident points, FlashAssign and update times from the light
+# event profile.
+OTHER_WORKLOADS = ["zipf", "splitd", "tiny", "f32large"]
+
+
+def time_workload(name, dev, steps=3, warmup=2):
+    import torch
+
+    import clustering_flashassign_b200 as fk
+    import synthdata
+    w = synthdata.WORKLOADS[name]
+    x, _, init = synthdata.make(w)
+
+    def as_torch(a):
+        t = torch.from_numpy(a)
+        return t.view(torch.bfloat16) if w.dtype == "bf16" else t
+
+    xd, initd = as_torch(x).to(dev), as_torch(init).to(dev)
+    ids = torch.empty((w.B, w.N), dtype=torch.int32, device=dev)
+    cen = torch.empty((w.B, w.K, w.d), dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        fk.fk_lloyd(xd, initd, w.iters, w.tol, ids, cen)
+    torch.cuda.synchronize(dev)
+    fk.fk_profile_read(reset=True)
+    fk.fk_profile_enable(2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    iters = 0
+    e0.record()
+    for _ in range(steps):
+        iters += fk.fk_lloyd(xd, initd, w.iters, w.tol, ids, cen)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    fk.fk_profile_enable(False)
+    prof = fk.fk_profile_read(reset=True)
+    ms = e0.elapsed_time(e1)
+    a_ms = prof["assign_ms"] / max(1, prof["assign_launches"])
+    flop = 2.0 * w.B * w.N * w.K * w.d
+    return {"shape": f"B={w.B} N={w.N} K={w.K} d={w.d} {w.dtype}", "iter_per_s": iters / (ms * 1e-3),
+            "assign_ms": a_ms, "assign_tflops": flop / (a_ms * 1e-3) / 1e12,
+            "update_ms": prof["update_ms"] / max(1, prof["update_calls"]), "iterations": iters}
 
 
 def timeline_summary(tl):
@@ -749,6 +799,8 @@ def main():
                     help="time the materialised-distance assign and the scatter-atomic update next to libfk")
     ap.add_argument("--no-baselines", action="store_true",
                     help="leave the two baseline timings out of the bench line")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="leave the timings of the other workloads out of the bench line")
     ap.add_argument("--workload", default="api", choices=["api", "tiny", "zipf", "splitd", "largen", "f32large"],
                     help="api is the benchmark; the others print their own line (largen: the 64 GiB "
                          "streamed workload)")
