@@ -173,7 +173,7 @@ int assign_f32_tc(Workspace *ws, const float *x, const float *c, const float *x3
 int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const void *cnx,
                        const float *xn, int B, long long N, int K, int d, int dtype, long long Kpad,
                        int32_t *ids, cudaStream_t s, uint32_t *hist = nullptr,
-                       const float *x3 = nullptr) {
+                       const float *x3 = nullptr, float *xn_out = nullptr) {
   PhaseTimer t(PH_ASSIGN, s);
   if (dtype == FK_F32) {
     if (use_tf32(K, d))
@@ -182,7 +182,7 @@ int do_assign_resident(Workspace *ws, const void *x, const void *cdt, const void
   }
   // 16-bit split-d tiles (128 x d x 2 bytes) stay in L2 across a tile's
   // chunks, so one work item per tile (no per-chunk merge) is the faster order
-  return launch_assign_tc(x, cdt, cnx, xn, dtype, B, N, K, d, Kpad, ids, ws->err, s, hist);
+  return launch_assign_tc(x, cdt, cnx, xn, dtype, B, N, K, d, Kpad, ids, ws->err, s, hist, nullptr, xn_out);
 }
 
 int read_shift(Workspace *ws, cudaStream_t s, float *out) {
@@ -602,10 +602,10 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
       cnx = ws->cn.p;
       if (max_iter > 1 && d <= 2 * kBlockK) {
         // the resident-tile assign ranks with ||x||^2 too; the points do not
-        // change, so their norms are computed once per call
+        // change, so the first assign stores the norms it computes from its
+        // shared tiles and the later ones read them
         FK_TRY(ensure(ws->xn, (size_t)B * N * sizeof(float)));
         xn = (float *)ws->xn.p;
-        FK_TRY(launch_point_norms(xdev, dtype, (long long)B * N, d, xn, s));
       }
     }
     FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cnx, ws->err, s));
@@ -646,7 +646,9 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
       return do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, out, s, hist, x3);
     };
     int cur = 0;
-    if (max_iter > 0) FK_TRY(assign(idbuf[0]));
+    if (max_iter > 0)  // the first assign computes the point norms and keeps them in xn
+      FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, nullptr, B, N, K, d, dtype, Kpad, idbuf[0], s, hist, x3,
+                                xn));
     for (int it = 0; it < max_iter; ++it) {
       FK_TRY(do_update(ws, xdev, idbuf[cur], B, N, K, d, dtype, cen_dev, nullptr, ch, cnx, Kpad, s, fuse));
       iters = it + 1;

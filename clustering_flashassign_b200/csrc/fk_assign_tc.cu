@@ -98,6 +98,7 @@ struct TcArgs {
   int nchunks;
   int kblocks;
   const float *xn;  // ||x||^2 per point (B, N), or NULL: computed from the shared tile
+  float *xn_out;    // nullable (resident, xn NULL): the computed norms are stored here too
   int32_t *ids;
   int *err;
   uint32_t idesc;
@@ -458,6 +459,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int q = 0; q < kTileM / 32; ++q) xn2[q] = s0[q] + s1[q];
+          if (a.xn_out) {  // kept for later assigns of the same points
+#pragma unroll
+            for (int q = 0; q < kTileM / 32; ++q) {
+              const int row = row0 + q * 32 + lane;
+              if (row < a.N) a.xn_out[(size_t)b * a.N + row] = xn2[q];
+            }
+          }
         }
         bool clamped = false;
 #pragma unroll
@@ -784,7 +792,7 @@ int launch_point_norms(const void *x, int dtype, long long rows, int d, float *x
 
 int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float *xn, int dtype,
                      int B, long long N, int K, int d, long long Kpad, int32_t *ids, int *err,
-                     cudaStream_t s, uint32_t *hist, unsigned long long *keys) {
+                     cudaStream_t s, uint32_t *hist, unsigned long long *keys, float *xn_out) {
   // K-blocks are 128-byte rows: 64 16-bit elements or 32 fp32 (read as tf32);
   // norm rows are 32 bytes: 16 or 8 elements
   const int blk = dtype == FK_F32 ? 32 : kBlockK;
@@ -805,6 +813,7 @@ int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float
   a.nchunks = (K + kChunkN - 1) / kChunkN;
   a.kblocks = (d + blk - 1) / blk;
   a.xn = xn;
+  a.xn_out = xn ? nullptr : xn_out;
   a.ids = ids;
   a.err = err;
   a.xg = x;

@@ -188,9 +188,12 @@ int launch_prep_ext_f32(const float *c, int B, int K, int d, long long Kpad, voi
 // (run_sort_prehist then skips its histogram kernel).
 int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float *xn, int dtype,
                      int B, long long N, int K, int d, long long Kpad, int32_t *ids, int *err,
-                     cudaStream_t s, uint32_t *hist = nullptr, unsigned long long *keys = nullptr);
+                     cudaStream_t s, uint32_t *hist = nullptr, unsigned long long *keys = nullptr,
+                     float *xn_out = nullptr);
 // keys: (B, N) zeroed scratch for the split-d variant's per-chunk work items
 // (left zeroed again); NULL keeps one work item per point tile.
+// xn_out (resident variant, xn NULL): the point norms computed from the shared
+// tiles are also stored there, (B, N) fp32, bit-identical to launch_point_norms.
 // xn[r] = ||x_r||^2 (fp32 accumulation) for `rows` rows of d 16-bit elements.
 int launch_point_norms(const void *x, int dtype, long long rows, int d, float *xn, cudaStream_t s);
 
