@@ -36,6 +36,7 @@ struct ChunkEvents {
   int buf;
 };
 std::vector<ChunkEvents> g_chunks;
+constexpr size_t kMaxTimelineChunks = 1 << 16;  // 4 events each; recording stops here until read
 }  // namespace
 
 int set_error(int status, const std::string &msg) {
@@ -271,13 +272,17 @@ int chunk_event(int which, long long chunk, int buf, cudaStream_t s) {
   if (g_prof_level != 3) return FK_OK;
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (which == 0) {
+    if (g_chunks.size() >= kMaxTimelineChunks) return FK_OK;  // the record is full until read
     ChunkEvents c;
     c.chunk = chunk;
     c.buf = buf;
     for (auto &e : c.ev) FK_CUDA(cudaEventCreate(&e));
+    for (auto &e : c.ev) FK_CUDA(cudaEventRecord(e, s));  // a chunk cut short still has four events
     g_chunks.push_back(c);
+    return FK_OK;
   }
-  if (g_chunks.empty() || g_chunks.back().chunk != chunk) return set_error(FK_EINVAL, "chunk events out of order");
+  // profiling turned on in the middle of a chunk, or a full record: not recorded
+  if (g_chunks.empty() || g_chunks.back().chunk != chunk) return FK_OK;
   FK_CUDA(cudaEventRecord(g_chunks.back().ev[which], s));
   return FK_OK;
 }

@@ -362,7 +362,9 @@ int fk_profile_enable(int on);
  * the compute stream: assign, sort and segment reduce of the chunk)}, times
  * in ms from the first chunk's copy begin.  Writes at most max_chunks rows to
  * out (host; NULL discards them) and their number to *rows (host, nullable),
- * synchronizes the recorded events and clears the record.  FK_EINVAL for
+ * synchronizes the recorded events and clears the record.  At most 65536
+ * chunks are kept between two reads (later ones are not recorded); a chunk
+ * whose copy began before level 3 was set is not recorded.  FK_EINVAL for
  * max_chunks < 0.  It measures the chunked host-to-device overlap
  * ("Flash-KMeans: Fast and Memory-Efficient Exact K-Means", Abstract:
  * chunked-stream overlap); an interface addition, the pages show no timeline.
