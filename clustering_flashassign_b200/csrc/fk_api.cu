@@ -495,7 +495,9 @@ int fk_lloyd_step_partial(const fk_shape *shape, const void *x, const float *xn,
     hist = (uint32_t *)ws->table.p;
     FK_CUDA(cudaMemsetAsync(hist, 0, hist_bytes, s));
   }
-  const float *xnr = (tc && d <= 2 * kBlockK) ? xn : nullptr;
+  // the resident assign ranks with the norms; the split-d one reads them for
+  // its far-point check
+  const float *xnr = tc ? xn : nullptr;
   FK_TRY(do_assign_resident(ws, x, centers_dt, cnx, xnr, B, N, K, d, dtype, Kpad, ids, s, hist));
   return do_partial(ws, x, ids, B, N, K, d, dtype, sums, counts, s, fuse);
 }
@@ -606,6 +608,12 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
         // shared tiles and the later ones read them
         FK_TRY(ensure(ws->xn, (size_t)B * N * sizeof(float)));
         xn = (float *)ws->xn.p;
+      } else if (max_iter > 0 && d > 2 * kBlockK) {
+        // the split-d assign's far-point check reads ||x||^2: one pass over
+        // the points per call instead of row reads in every assign
+        FK_TRY(ensure(ws->xn, (size_t)B * N * sizeof(float)));
+        xn = (float *)ws->xn.p;
+        FK_TRY(launch_point_norms(xdev, dtype, (long long)B * N, d, xn, s));
       }
     }
     FK_TRY(launch_init_centers(init_dev, dtype, B, K, d, Kpad, cen_dev, ch, cnx, ws->err, s));
@@ -646,9 +654,9 @@ int fk_lloyd(const fk_shape *shape, const void *x, const void *init_centers, int
       return do_assign_resident(ws, xdev, cassign, cnx, xn, B, N, K, d, dtype, Kpad, out, s, hist, x3);
     };
     int cur = 0;
-    if (max_iter > 0)  // the first assign computes the point norms and keeps them in xn
-      FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, nullptr, B, N, K, d, dtype, Kpad, idbuf[0], s, hist, x3,
-                                xn));
+    if (max_iter > 0)  // resident: the first assign computes the point norms and keeps them in xn
+      FK_TRY(do_assign_resident(ws, xdev, cassign, cnx, d > 2 * kBlockK ? xn : nullptr, B, N, K, d, dtype, Kpad,
+                                idbuf[0], s, hist, x3, xn));
     for (int it = 0; it < max_iter; ++it) {
       FK_TRY(do_update(ws, xdev, idbuf[cur], B, N, K, d, dtype, cen_dev, nullptr, ch, cnx, Kpad, s, fuse));
       iters = it + 1;

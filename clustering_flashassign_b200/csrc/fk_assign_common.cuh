@@ -30,6 +30,17 @@ __device__ __forceinline__ float key_hi(float key) {
 // holds for x = 0.
 constexpr float kFarRatioHalf = 8.f;
 
+// The exact-value paths (split-d) rank by v = x.c - ||c||^2 / 2 =
+// (||x||^2 - ||x - c||^2) / 2 in fp32.  Far from the origin compared with
+// ||x||, the fp32 rounding of v is set by ||c||^2 and can exceed the near-tie
+// band: a row with ||x - c||^2 > 64 ||x||^2, i.e. -2 v > 63 ||x||^2, is
+// re-ranked exactly.  Only rows with v < 0 (nearest distance above ||x||^2)
+// can qualify, so ||x||^2 is read (or computed) for those alone.  Below the
+// threshold ||c|| <= 9 ||x||, and the worst-case fp32 error of v (about
+// (d / 16) u ||x|| ||c|| for the MMA's accumulation) stays inside the band for
+// d up to a few thousand; typical errors grow as sqrt(d).
+constexpr float kFarRatioExactM1 = 63.f;
+
 __device__ __forceinline__ double widen_lo(uint32_t v, __half) {
   return (double)__half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu)));
 }
@@ -43,6 +54,32 @@ __device__ __forceinline__ double widen_hi(uint32_t v, __nv_bfloat16) {
   return (double)__uint_as_float(v & 0xFFFF0000u);
 }
 
+// Partial ||x||^2 (fp32) of one 16-bit row, summed in 64-element blocks until
+// kFarRatioExactM1 times it reaches `lim2` (= -2 v): the full norm when the row
+// is far, else a partial sum that already rules the row out (most rows stop
+// after one block).  d % 8 == 0, 16-byte aligned rows.
+template <typename T>
+__device__ __forceinline__ float row_norm2_upto(const T *__restrict__ x, int d, float lim2) {
+  const uint4 *xr = reinterpret_cast<const uint4 *>(x);
+  const int n = d / 8;
+  float s = 0.f;
+  for (int j0 = 0; j0 < n && kFarRatioExactM1 * s < lim2; j0 += 8) {
+    uint4 v[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) v[t] = j0 + t < n ? __ldg(xr + j0 + t) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const uint32_t w[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float lo = (float)widen_lo(w[q], T()), hi = (float)widen_hi(w[q], T());
+        s = fmaf(lo, lo, s);
+        s = fmaf(hi, hi, s);
+      }
+    }
+  }
+  return s;
+}
 
 // Exact nearest centroid of one point, computed by the whole warp: lane l
 // takes centroids l, l + 32, ... and sums (x_j - c_kj)^2 over j in fp64 (the

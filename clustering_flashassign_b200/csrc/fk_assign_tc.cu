@@ -63,7 +63,13 @@
 //               With a keys buffer every (tile, chunk) pair is its own work
 //               item, consecutive CTAs taking one tile's chunks so they share
 //               its reads in L2; the chunks merge by a 64-bit atomicMax per
-//               point and k_keys_to_ids writes the ids.
+//               point and k_keys_to_ids writes the ids.  For 16-bit points
+//               the fp32 rounding of acc is set by ||c||^2, so a point whose
+//               nearest squared distance exceeds 64 ||x||^2 (||x||^2 from the
+//               caller's precomputed norms, else read from its row) is
+//               re-ranked exactly as above; when it is flagged in its best
+//               chunk it is flagged in every chunk, so every work item
+//               reports the exact id.
 // Every role waits by polling its mbarriers without suspending (a suspended
 // thread resumes hundreds of cycles after the phase completes, and the
 // per-chunk hand-offs between the roles are on the tensor core's critical
@@ -632,6 +638,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           // far-point check (see the header): flagged rows of this warp are
           // re-ranked one after another by the whole warp
           unsigned flagged = __ballot_sync(0xffffffffu, row < a.N && -val > kFarRatioHalf * o.z);
+          while (flagged) {
+            const int src = __ffs(flagged) - 1;
+            flagged &= flagged - 1;
+            const int r = row0 + quad * 32 + src;
+            const T *xrow = static_cast<const T *>(a.xg) + ((size_t)b * a.N + r) * a.d;
+            const T *cb = static_cast<const T *>(a.cg) + (size_t)b * a.K * a.d;
+            const int k = exact_argmin_warp<T>(xrow, cb, a.K, a.d, lane);
+            if (lane == src) idx = k;
+          }
+        }
+        if constexpr (!RESIDENT && sizeof(T) == 2) {
+          // far-point check of the exact-value path (fk_assign_common.cuh):
+          // rows with v < 0 take ||x||^2 from the precomputed norms, else
+          // sum their row in global memory until it rules them out, and
+          // those far from every centroid compared with it are re-ranked
+          // exactly
+          const bool maybe = row < a.N && val < 0.f;
+          float xn2 = 0.f;
+          if (maybe)
+            xn2 = a.xn ? __ldg(a.xn + (size_t)b * a.N + row)
+                       : row_norm2_upto<T>(static_cast<const T *>(a.xg) + ((size_t)b * a.N + row) * a.d, a.d,
+                                           -2.f * val);
+          unsigned flagged = __ballot_sync(0xffffffffu, maybe && kFarRatioExactM1 * xn2 < -2.f * val);
           while (flagged) {
             const int src = __ffs(flagged) - 1;
             flagged &= flagged - 1;

@@ -230,7 +230,9 @@ int fk_init_centers(const void *init, int B, int K, int d, int dtype, float *cen
  *               (then streamed in chunks of opts->chunk_points, double-
  *               buffered, as fk_lloyd's streamed mode).
  *   xn          nullable (B, N) fp32, device: fk_point_norms of x (used for
- *               device-resident fp16 / bf16 points with d <= 128; else ignored).
+ *               device-resident fp16 / bf16 points: with d <= 128 the assign
+ *               ranks with them, with d > 128 its far-point check reads them
+ *               instead of re-reading rows; else ignored).
  *   centers_dt  (B, K, d) in dtype, device: the centroids to assign against
  *               (for fp32 the fp32 centroids themselves).
  *   ids         (B, N) int32 out, device.

@@ -18,6 +18,15 @@ in fp64.  These inputs put every point there:
   centroids of equal norm (the lowest index must win) and one of a norm one
   step smaller at a higher index.
 
+The split-d assign (16-bit points, d > 128) ranks by the exact value
+v = x.c - ||c||^2 / 2 in fp32, whose rounding is set by ||c||^2: with points
+near the origin and centroids of norm ~16, pairs one step apart give v gaps
+of about one fp32 step of v, above the near-tie band 1e-3 ||x||^2.  The
+kernel re-ranks rows whose nearest distance exceeds 64 ||x||^2 in fp64; K is
+chosen to span several 256-centroid chunks, so both the per-chunk work items
+(fk_assign, fk_lloyd_step_partial) and the whole-tile items
+(fk_assign_noalloc) are covered.
+
 Each case runs through fk_assign (point norms from the shared tile),
 fk_lloyd_step_partial with precomputed norms, and fk_assign_noalloc.
 """
@@ -53,6 +62,20 @@ def far_pairs(B, N, d, dtype, seed):
     # is 1e-3 ||x||^2 ~ 2e-4 and 2^-15 of the distance 1e-3 or more
     scale, c0 = (1.0, 0.75) if dtype == "f16" else (2.0, 0.375)
     v = _round16(scale * rng.standard_normal((B, K // 2, d)), dtype)
+    v[..., 0] = _round16(np.full((B, K // 2), c0), dtype)
+    c = np.repeat(v, 2, axis=1)
+    c[:, 1::2, 0] = _step(c[:, 1::2, 0], dtype)
+    return x, c
+
+
+def far_pairs_splitd(B, N, K, d, dtype, seed):
+    rng = np.random.default_rng(seed)
+    # fp16: a step at 0.125 is 2^-14, a v gap of about 2^-15 next to v ~ -128
+    # (fp32 step 2^-16 there); bf16: a step at 2^-5 is 2^-13, a v gap of
+    # about 2^-18; the band is 1e-3 ||x||^2 ~ 6e-6 (x scale 0.005 / 0.004)
+    xs, c0 = (0.005, 0.125) if dtype == "f16" else (0.004, 0.03125)
+    x = _round16(xs * rng.standard_normal((B, N, d)), dtype)
+    v = _round16(rng.standard_normal((B, K // 2, d)), dtype)
     v[..., 0] = _round16(np.full((B, K // 2), c0), dtype)
     c = np.repeat(v, 2, axis=1)
     c[:, 1::2, 0] = _step(c[:, 1::2, 0], dtype)
@@ -114,6 +137,25 @@ def test_far_points_with_close_pairs_take_the_nearer_centroid(B, N, d, dtype):
     # their top-2 gap lies above the band but below 2^-15 of the distance, and
     # the nearer centroid is the higher (odd) index of its pair
     window = (gap > ID_GAP_REL * xn) & (gap < 2.0 ** -15 * dmin) & (dmin > 16 * xn)
+    assert window.mean() > 0.9
+    assert (ref[window] % 2 == 1).all()
+    for name, g in _run_all(x, c, dtype).items():
+        assert check_ids(g, x, dtype, chat, ref, gap) == 0, name
+        assert np.array_equal(g, ref), name
+
+
+@pytest.mark.parametrize("B,N,K,d,dtype", [(2, 1500, 600, 256, "f16"), (2, 1500, 600, 256, "bf16"),
+                                           (1, 900, 64, 320, "f16")])
+def test_splitd_far_points_with_close_pairs_take_the_nearer_centroid(B, N, K, d, dtype):
+    x, c = far_pairs_splitd(B, N, K, d, dtype, seed=5 + d)
+    chat = synthdata.to_f64(c, dtype)
+    ref, gap, dmin = oracle.assign(x, dtype, chat)
+    xn = xnorm2(x, dtype)
+    # every point is far (> 64 ||x||^2), its top-2 gap lies above the band,
+    # half of it (the v gap) within two fp32 steps of v ~ -dmin / 2, and the
+    # nearer centroid is the odd one of its pair
+    ulp_v = np.spacing((dmin / 2).astype(np.float32)).astype(np.float64)
+    window = (gap > ID_GAP_REL * xn) & (gap / 2 < 2 * ulp_v) & (dmin > 64 * xn)
     assert window.mean() > 0.9
     assert (ref[window] % 2 == 1).all()
     for name, g in _run_all(x, c, dtype).items():
