@@ -28,12 +28,15 @@
 //   warp 10     (resident variant) ||x||^2 of each point tile from the shared
 //               copy, written as the tile's norm rows,
 //   warp 11     (resident variant) the point tiles (128 x d), one tile ahead.
-// The MMA thread is the pipeline's serial point, so in the resident variant
-// it waits on one barrier per chunk and commits once: the producer, after
-// issuing a chunk's copies, also waits for the chunk's accumulator to be free
-// (and, for a tile's first chunk, for the tile's norm rows) and then arrives
-// on the stage's full barrier a second time; the chunk's single commit frees
-// the stage and tells the epilogue that the accumulator is complete.
+// In the resident variant the MMA thread waits per chunk for its accumulator
+// (released by the epilogue) and for the stage, and commits once to the
+// stage's empty barrier: the stage is free and the epilogue may read the
+// accumulator.  With two K-blocks it also commits after K-block 0, so the
+// producer refills that half of the stage half a chunk earlier; the producer
+// waits for nothing else and runs ahead as far as the stages allow.  The
+// centroids' norm rows are stored pre-swizzled (fk_centroids.cu) and arrive
+// by one bulk copy per chunk: the TMA unit moves tiles row by row, and 256
+// rows of 32 bytes cost it about as much as 256 rows of 128 bytes.
 // Two variants, picked by d:
 //   resident X (d <= 128): the point tile stays in shared memory for all K
 //               chunks (double-buffered across tiles); only centroids stream.
@@ -119,6 +122,9 @@ struct TcArgs {
   // split-d only, optional: per-point packed (value, index) keys; then every
   // (tile, chunk) pair is its own work item and chunks merge by atomicMax
   unsigned long long *keys;
+  // the centroids' extension rows: per (batch, chunk) the kBExtBytes
+  // shared-memory image of the chunk's 32-byte-swizzled norm rows
+  const uint8_t *cnx;
 };
 
 // (value, index) as one 64-bit key whose unsigned order is: larger value
@@ -146,8 +152,8 @@ struct Layout {
   static constexpr uint32_t kBarOff = kStagesOff + STAGES * kStageBytes;
   // barriers: full[S], empty[S], efull[E], eempty[E], xfull[2], xempty[2],
   //           xnfull[2], accfull[2], accempty[2], mfull[2], mempty[2], drain,
-  //           xnfree[2]
-  static constexpr int kNumBars = 2 * STAGES + 2 * kExtSlots + 17;
+  //           xnfree[2], kbfree[S]
+  static constexpr int kNumBars = 3 * STAGES + 2 * kExtSlots + 17;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag
   static constexpr uint32_t kMergeOff = (kMiscOff + 16 + 15) / 16 * 16;
   // resident: ||x||^2 of the rows of the two point-tile buffers, for the
@@ -184,7 +190,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 template <typename T, bool RESIDENT, int KB, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     k_flash_assign(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmc,
-                   const __grid_constant__ CUtensorMap tme, const TcArgs a) {
+                   const TcArgs a) {
   using L = Layout<RESIDENT, KB, STAGES>;
   constexpr int kBlockE = 128 / (int)sizeof(T);  // elements per 128-byte K-block row
   static_assert(!RESIDENT || sizeof(T) == 2, "the resident-tile variant is for 16-bit points");
@@ -210,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto mempty = [&](int i) { return bar0 + 8u * (kB2 + 12 + i); };
   const uint32_t drain = bar0 + 8u * (kB2 + 14);
   auto xnfree = [&](int i) { return bar0 + 8u * (kB2 + 15 + i); };
+  auto kbfree = [&](int s) { return bar0 + 8u * (kB2 + 17 + s); };
   float *xnorm_s = reinterpret_cast<float *>(smem + L::kXnOff);  // [2][kTileM], resident only
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
@@ -219,11 +226,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      // resident: the producer arrives twice, once with the copies' byte count
-      // and once when the chunk's accumulator (and, for a tile's first chunk,
-      // the tile's norm rows) are free to use
-      mbar_init(full(s), RESIDENT ? 2 : 1);
+      mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
+      mbar_init(kbfree(s), 1);  // resident, two K-blocks: K-block 0 of the stage read
     }
     for (int e = 0; e < kExtSlots; ++e) {
       mbar_init(efull(e), 1);
@@ -247,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmx);
     prefetch_tensormap(&tmc);
-    prefetch_tensormap(&tme);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -286,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t f = 0, e = 0, u = 0;  // stages, ext rows, tiles done
+      uint32_t f = 0, e = 0;  // stages, ext rows
       bool ok = true;
       for (int task = blockIdx.x; ok && task < ntask; task += gridDim.x) {
         const int tile = task_tile(task);
@@ -295,28 +299,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = chunk_lo(task); ok && c < chunk_hi(task); ++c) {
           if (RESIDENT) {  // the whole chunk and its norm rows in one stage
             // empty(s) is committed once per chunk by the MMA thread: the
-            // stage is free and the epilogue may read the chunk's accumulator
+            // stage is free and the epilogue may read the chunk's accumulator.
+            // With two K-blocks, K-block 0 is refilled as soon as the chunk
+            // STAGES back has read it (kbfree), half a chunk earlier; its
+            // bytes are expected before the copy and the one arrival comes
+            // with the rest, so the phase cannot complete early.
             const int s = f % STAGES;
-            if (!mbar_wait_spin(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
+            const uint32_t par = ((f / STAGES) & 1) ^ 1;
             const uint32_t dst = st_base + s * L::kStageBytes;
-            mbar_arrive_expect_tx(full(s), L::kStageBytes);
-            for (int kb = 0; kb < KB; ++kb)
+            if constexpr (KB == 2) {
+              if (!mbar_wait_spin(kbfree(s), par, abort_flag, a.err)) { ok = false; break; }
+              mbar_expect_tx(full(s), kCBlockBytes);
+              tma_load_3d(&tmc, dst, full(s), 0, c * kChunkN, b);
+            }
+            if (!mbar_wait_spin(empty(s), par, abort_flag, a.err)) {
+              if (KB == 2) {  // let the phase complete as K-block 0 lands; the tail drains it
+                mbar_arrive(full(s));
+                ++f;
+              }
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(full(s), L::kStageBytes - (KB == 2 ? kCBlockBytes : 0u));
+            for (int kb = KB == 2 ? 1 : 0; kb < KB; ++kb)
               tma_load_3d(&tmc, dst + kb * kCBlockBytes, full(s), kb * kBlockE, c * kChunkN, b);
-            tma_load_3d(&tme, dst + KB * kCBlockBytes, full(s), 0, c * kChunkN, b);
-            // The MMA thread waits on full(s) alone: this thread takes the
-            // other waits of the chunk off its path between two chunks.
-            bool ready = true;
-            if (c == 0)  // the tile's point norm rows are written (so its copy landed too)
-              ready = mbar_wait_spin(xnfull(u & 1), (u >> 1) & 1, abort_flag, a.err);
-            ready = ready && mbar_wait_spin(accempty(f & 1), ((f >> 1) & 1) ^ 1, abort_flag, a.err);
-            mbar_arrive(full(s));  // also when aborting, so the phase completes as the copies land
+            bulk_load(dst + KB * kCBlockBytes, a.cnx + ((size_t)b * a.nchunks + c) * kBExtBytes, kBExtBytes,
+                      full(s));
             ++f;
-            if (!ready) { ok = false; break; }
           } else {  // this chunk's centroid norm rows (used by the chunk's last MMA step)
             const int es = e % kExtSlots;
             if (!mbar_wait_spin(eempty(es), ((e / kExtSlots) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
             mbar_arrive_expect_tx(efull(es), kBExtBytes);
-            tma_load_3d(&tme, bext_base + es * kBExtBytes, efull(es), 0, c * kChunkN, b);
+            bulk_load(bext_base + es * kBExtBytes, a.cnx + ((size_t)b * a.nchunks + c) * kBExtBytes, kBExtBytes,
+                      efull(es));
             ++e;
           }
           for (int kb = 0; !RESIDENT && kb < kblocks; ++kb) {
@@ -329,7 +344,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++f;
           }
         }
-        ++u;
       }
       // tail: make every issued copy and every release of a buffer land before exit
       const bool aborted = *abort_flag != 0;
@@ -346,20 +360,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int task = blockIdx.x; ok && task < ntask; task += gridDim.x) {
         int xb = 0;
-        if (RESIDENT) {
+        if (RESIDENT) {  // the point tile and its norm rows
           xb = g & 1;
           if (!mbar_wait_spin(xfull(xb), (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+          if (!mbar_wait_spin(xnfull(xb), (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
         }
         const uint32_t a_ext = aext_base + (RESIDENT ? xb * kAExtBytes : 0u);
         for (int c = chunk_lo(task); ok && c < chunk_hi(task); ++c) {
           const int ab = h & 1;
           if (RESIDENT) {
-            // full(s) also stands for the free accumulator and the tile's norm
-            // rows (the producer's second arrival); one commit per chunk to
-            // empty(s) frees the stage and hands the accumulator to the epilogue
+            // the accumulator is free (the epilogue's release of the chunk two
+            // back) and the stage has landed; one commit per chunk to empty(s)
+            // frees the stage and hands the accumulator to the epilogue
             const uint32_t d_tmem = tmem + ab * kChunkN;
             const int s = f % STAGES;
+            if (!mbar_wait_spin(accempty(ab), ((h >> 1) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
             if (!mbar_wait_spin(full(s), (f / STAGES) & 1, abort_flag, a.err)) { ok = false; break; }
             tc_fence_after();
             const uint32_t stage = st_base + s * L::kStageBytes;
@@ -371,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int k = 0; k < kBlockK / 16; ++k)
                 mma_t<T>(d_tmem, desc_k_sw128(a_addr + k * 32), desc_k_sw128(b_addr + k * 32), a.idesc,
                         (kb | k) != 0 ? 1u : 0u);
+              if (KB == 2 && kb == 0) mma_commit(kbfree(s));  // K-block 0 may be refilled
             }
             // the norm step: acc += A_ext . B_ext (fk_norms.cuh)
             mma_t<T>(d_tmem, desc_k_sw32(a_ext), desc_k_sw32(stage + KB * kCBlockBytes), a.idesc, 1u);
@@ -790,26 +807,24 @@ int encode_3d(CUtensorMap *map, const void *base, int dtype, int inner, long lon
 }
 
 template <typename T, bool RESIDENT, int KB, int STAGES>
-int launch_variant(const CUtensorMap &tmx, const CUtensorMap &tmc, const CUtensorMap &tme,
-                   const TcArgs &a, int grid, cudaStream_t s) {
+int launch_variant(const CUtensorMap &tmx, const CUtensorMap &tmc, const TcArgs &a, int grid, cudaStream_t s) {
   using L = Layout<RESIDENT, KB, STAGES>;
   FK_TRY(set_smem_limit((const void *)k_flash_assign<T, RESIDENT, KB, STAGES>, (int)L::kAlloc));
   FK_CUDA(launch_pdl(k_flash_assign<T, RESIDENT, KB, STAGES>, dim3(grid), dim3(kThreads), L::kAlloc, s, tmx, tmc,
-                     tme, a));
+                     a));
   FK_TRY(launched());
   FK_CUDA(cudaGetLastError());
   return FK_OK;
 }
 
 template <typename T>
-int launch_typed(const CUtensorMap &tmx, const CUtensorMap &tmc, const CUtensorMap &tme,
-                 const TcArgs &a, int grid, cudaStream_t s) {
+int launch_typed(const CUtensorMap &tmx, const CUtensorMap &tmc, const TcArgs &a, int grid, cudaStream_t s) {
   // resident stages hold whole chunks: 4 x 40 KB (d <= 64) or 2 x 72 KB (d <= 128)
   if constexpr (sizeof(T) == 2) {
-    if (a.kblocks == 1) return launch_variant<T, true, 1, 4>(tmx, tmc, tme, a, grid, s);
-    if (a.kblocks == 2) return launch_variant<T, true, 2, 2>(tmx, tmc, tme, a, grid, s);
+    if (a.kblocks == 1) return launch_variant<T, true, 1, 4>(tmx, tmc, a, grid, s);
+    if (a.kblocks == 2) return launch_variant<T, true, 2, 2>(tmx, tmc, a, grid, s);
   }
-  return launch_variant<T, false, 1, 4>(tmx, tmc, tme, a, grid, s);
+  return launch_variant<T, false, 1, 4>(tmx, tmc, a, grid, s);
 }
 
 }  // namespace
@@ -823,14 +838,16 @@ int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float
                      int B, long long N, int K, int d, long long Kpad, int32_t *ids, int *err,
                      cudaStream_t s, uint32_t *hist, unsigned long long *keys, float *xn_out) {
   // K-blocks are 128-byte rows: 64 16-bit elements or 32 fp32 (read as tf32);
-  // norm rows are 32 bytes: 16 or 8 elements
+  // norm rows are 32 bytes (16 or 8 elements), stored per 256-row chunk as
+  // the shared-memory image of the swizzled tile and moved by bulk copies
   const int blk = dtype == FK_F32 ? 32 : kBlockK;
-  const int ext = dtype == FK_F32 ? kExtF32 : kExt;
-  CUtensorMap tmx, tmc, tme;
+  if (Kpad != (long long)(K + kChunkN - 1) / kChunkN * kChunkN || (reinterpret_cast<uintptr_t>(cnx) & 15u))
+    return set_error(FK_EINVAL, "extension rows: Kpad must be K rounded up to the chunk, 16-byte aligned");
+  CUtensorMap tmx, tmc;
   FK_TRY(encode_3d(&tmx, x, dtype, d, N, B, blk, kTileM, CU_TENSOR_MAP_SWIZZLE_128B));
   FK_TRY(encode_3d(&tmc, ch, dtype, d, K, B, blk, kChunkN, CU_TENSOR_MAP_SWIZZLE_128B));
-  FK_TRY(encode_3d(&tme, cnx, dtype, ext, Kpad, B, ext, kChunkN, CU_TENSOR_MAP_SWIZZLE_32B));
   TcArgs a;
+  a.cnx = static_cast<const uint8_t *>(cnx);
   a.N = (int)N;
   a.K = K;
   a.hist = hist;
@@ -857,9 +874,9 @@ int launch_assign_tc(const void *x, const void *ch, const void *cnx, const float
   const long long tasks = a.keys ? total * a.nchunks : total;
   int grid = num_sms();
   if (tasks < grid) grid = (int)tasks;
-  if (dtype == FK_F32) FK_TRY(launch_typed<float>(tmx, tmc, tme, a, grid, s));
-  else if (dtype == FK_BF16) FK_TRY(launch_typed<__nv_bfloat16>(tmx, tmc, tme, a, grid, s));
-  else FK_TRY(launch_typed<__half>(tmx, tmc, tme, a, grid, s));
+  if (dtype == FK_F32) FK_TRY(launch_typed<float>(tmx, tmc, a, grid, s));
+  else if (dtype == FK_BF16) FK_TRY(launch_typed<__nv_bfloat16>(tmx, tmc, a, grid, s));
+  else FK_TRY(launch_typed<__half>(tmx, tmc, a, grid, s));
   if (!a.keys) return FK_OK;
   const long long n = (long long)B * N;
   long long blocks = (n + 255) / 256;

@@ -47,15 +47,19 @@ constexpr int kWarpsPerBlock = 8;
 
 // Writes the tensor-core extension row of one centroid (see fk_norms.cuh);
 // rows past K get the sentinel row.  A norm beyond the fp16 digits' range is
-// recorded as DEV_RANGE in the device error word.
+// recorded as DEV_RANGE in the device error word.  The rows are stored as the
+// shared-memory image of a 32-byte-swizzled K-major tile (the two 16-byte
+// halves of row w swap places when bit 2 of w is set), so the assign moves a
+// chunk's 256 rows with one untiled bulk copy.
 template <typename T>
 __device__ __forceinline__ void store_ext(T *cnx, long long w, bool real, float cn, int *err) {
   if constexpr (sizeof(T) == 2) {
     alignas(16) T row[kExt];
     if (ext_centroid_row<T>(cn, real, row) && err) atomicCAS(err, DEV_OK, DEV_RANGE);
     uint4 *dst = reinterpret_cast<uint4 *>(cnx + (size_t)w * kExt);
-    dst[0] = *reinterpret_cast<const uint4 *>(&row[0]);
-    dst[1] = *reinterpret_cast<const uint4 *>(&row[8]);
+    const int flip = (int)((w >> 2) & 1);
+    dst[flip] = *reinterpret_cast<const uint4 *>(&row[0]);
+    dst[flip ^ 1] = *reinterpret_cast<const uint4 *>(&row[8]);
   } else {
     (void)cnx; (void)w; (void)real; (void)cn; (void)err;
   }

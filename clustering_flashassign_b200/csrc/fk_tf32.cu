@@ -50,11 +50,12 @@ __global__ void __launch_bounds__(256) k_prep_ext_f32(const float *__restrict__ 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   }
-  if (lane == 0) {
+  if (lane == 0) {  // stored pre-swizzled, like the 16-bit rows (fk_centroids.cu)
     alignas(16) float row[kExtF32];
     ext_centroid_row_f32(s, k < K, row);
-    cnx[2 * w] = *reinterpret_cast<const float4 *>(&row[0]);
-    cnx[2 * w + 1] = *reinterpret_cast<const float4 *>(&row[4]);
+    const int flip = (int)((w >> 2) & 1);
+    cnx[2 * w + flip] = *reinterpret_cast<const float4 *>(&row[0]);
+    cnx[2 * w + (flip ^ 1)] = *reinterpret_cast<const float4 *>(&row[4]);
   }
 }
 
