@@ -151,9 +151,9 @@ struct Layout {
       RESIDENT ? KB * kCBlockBytes + kBExtBytes : kXBlockBytes + kCBlockBytes;
   static constexpr uint32_t kBarOff = kStagesOff + STAGES * kStageBytes;
   // barriers: full[S], empty[S], efull[E], eempty[E], xfull[2], xempty[2],
-  //           xnfull[2], accfull[2], accempty[2], mfull[2], mempty[2], drain,
+  //           xnfull[2], accfull[2], accempty[2], mfull[4], mempty[4], drain,
   //           xnfree[2], kbfree[S]
-  static constexpr int kNumBars = 3 * STAGES + 2 * kExtSlots + 17;
+  static constexpr int kNumBars = 3 * STAGES + 2 * kExtSlots + 21;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag
   static constexpr uint32_t kMergeOff = (kMiscOff + 16 + 15) / 16 * 16;
   // resident: ||x||^2 of the rows of the two point-tile buffers, for the
@@ -212,11 +212,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto xnfull = [&](int i) { return bar0 + 8u * (kB2 + 4 + i); };
   auto accfull = [&](int i) { return bar0 + 8u * (kB2 + 6 + i); };
   auto accempty = [&](int i) { return bar0 + 8u * (kB2 + 8 + i); };
-  auto mfull = [&](int i) { return bar0 + 8u * (kB2 + 10 + i); };
-  auto mempty = [&](int i) { return bar0 + 8u * (kB2 + 12 + i); };
-  const uint32_t drain = bar0 + 8u * (kB2 + 14);
-  auto xnfree = [&](int i) { return bar0 + 8u * (kB2 + 15 + i); };
-  auto kbfree = [&](int s) { return bar0 + 8u * (kB2 + 17 + s); };
+  auto mfull = [&](int q) { return bar0 + 8u * (kB2 + 10 + q); };   // per TMEM lane quadrant
+  auto mempty = [&](int q) { return bar0 + 8u * (kB2 + 14 + q); };
+  const uint32_t drain = bar0 + 8u * (kB2 + 18);
+  auto xnfree = [&](int i) { return bar0 + 8u * (kB2 + 19 + i); };
+  auto kbfree = [&](int s) { return bar0 + 8u * (kB2 + 21 + s); };
   float *xnorm_s = reinterpret_cast<float *>(smem + L::kXnOff);  // [2][kTileM], resident only
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
@@ -237,12 +237,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(xfull(i), 1);
       mbar_init(xempty(i), 1);
-      mbar_init(xnfull(i), 1);
+      mbar_init(xnfull(i), 2);  // the norm and loader warps' halves
       mbar_init(accfull(i), 1);
       mbar_init(accempty(i), kEpiWarps);
-      mbar_init(mfull(i), kEpiWarps / 2);
-      mbar_init(mempty(i), kEpiWarps / 2);
+
       mbar_init(xnfree(i), kEpiWarps / 2);
+    }
+    for (int q = 0; q < 4; ++q) {  // the two warps of a lane quadrant hand over their halves
+      mbar_init(mfull(q), 1);
+      mbar_init(mempty(q), 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -437,42 +440,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_drain(drain, 0, a.err);
     }
     __syncwarp();
-  } else if (warp == kNormWarp) {
-    // ------------------------------------------------------------ point norms
+  } else if (warp == kNormWarp || warp == kLoadWarp) {
+    // ------------------------------------------------------------ point tiles and norms
+    // (resident) The loader's lane 0 requests tile g into the buffer of tile
+    // g - 2 as soon as that tile's MMAs are done, a whole tile ahead of its
+    // use.  ||x||^2 of each tile (the point-side norm rows, and the norms for
+    // the epilogue's far-point check) is split between the two warps, rows
+    // 0..63 here and 64..127 in the loader, so a tile whose norms are summed
+    // from its shared copy is ready in half the time.
+    uint32_t issued_tiles = 0;  // loader lane 0: tiles requested
     if constexpr (RESIDENT) {
-      bool ok = true;
+      constexpr int kQ = kTileM / 64;  // 32-row groups per warp
+      const bool loader = warp == kLoadWarp;
+      const int q0 = loader ? kQ : 0;
       uint32_t g = 0;
-      for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x, ++g) {
+      for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++g) {
         const int xb = g & 1;
         const int b = tile / a.tiles_per_batch;
         const int row0 = (tile % a.tiles_per_batch) * kTileM;
-        float xn2[kTileM / 32];
+        if (loader) {
+          int issued = 1;
+          if (lane == 0) {
+            issued = mbar_wait_spin(xempty(xb), ((g >> 1) & 1) ^ 1, abort_flag, a.err) ? 1 : 0;
+            if (issued) {
+              mbar_arrive_expect_tx(xfull(xb), KB * kXBlockBytes);
+              for (int kb = 0; kb < KB; ++kb)
+                tma_load_3d(&tmx, x_base + (xb * KB + kb) * kXBlockBytes, xfull(xb), kb * kBlockE, row0, b);
+            }
+          }
+          issued = __shfl_sync(0xffffffffu, issued, 0);
+          if (!issued) break;
+          if (lane == 0) ++issued_tiles;
+        }
+        float xn2[kQ];
         if (a.xn) {  // issued before the wait: the loads overlap it
 #pragma unroll
-          for (int q = 0; q < kTileM / 32; ++q) {
-            const int row = row0 + q * 32 + lane;
+          for (int q = 0; q < kQ; ++q) {
+            const int row = row0 + (q0 + q) * 32 + lane;
             xn2[q] = row < a.N ? __ldg(a.xn + (size_t)b * a.N + row) : 0.f;
           }
         }
         if (!warp_wait(xfull(xb), (g >> 1) & 1, abort_flag, a.err, lane)) break;
         if (!a.xn) {
-          // lane l sums rows l, l+32, l+64, l+96 of the swizzled tile (16-byte
-          // chunk j of row r sits at chunk j ^ (r & 7); r & 7 == l & 7 here)
-          float s0[kTileM / 32], s1[kTileM / 32];
+          // lane l sums rows l + 32 q of the swizzled tile (16-byte chunk j of
+          // row r sits at chunk j ^ (r & 7); r & 7 == l & 7 here)
+          float s0[kQ], s1[kQ];
 #pragma unroll
-          for (int q = 0; q < kTileM / 32; ++q) s0[q] = s1[q] = 0.f;
+          for (int q = 0; q < kQ; ++q) s0[q] = s1[q] = 0.f;
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) {
-            const uint8_t *blk = smem + (xb * KB + kb) * kXBlockBytes + lane * 128;
+            const uint8_t *blk = smem + (xb * KB + kb) * kXBlockBytes + (q0 * 32 + lane) * 128;
 #pragma unroll 2
             for (int j = 0; j < 8; ++j) {
               const int off = (j ^ (lane & 7)) << 4;
-              uint4 v[kTileM / 32];
+              uint4 v[kQ];
 #pragma unroll
-              for (int q = 0; q < kTileM / 32; ++q)
-                v[q] = *reinterpret_cast<const uint4 *>(blk + q * 32 * 128 + off);
+              for (int q = 0; q < kQ; ++q) v[q] = *reinterpret_cast<const uint4 *>(blk + q * 32 * 128 + off);
 #pragma unroll
-              for (int q = 0; q < kTileM / 32; ++q) {
+              for (int q = 0; q < kQ; ++q) {
                 sq2_acc<T>(v[q].x, s0[q], s1[q]);
                 sq2_acc<T>(v[q].y, s0[q], s1[q]);
                 sq2_acc<T>(v[q].z, s0[q], s1[q]);
@@ -481,21 +506,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
 #pragma unroll
-          for (int q = 0; q < kTileM / 32; ++q) xn2[q] = s0[q] + s1[q];
+          for (int q = 0; q < kQ; ++q) xn2[q] = s0[q] + s1[q];
           if (a.xn_out) {  // kept for later assigns of the same points
 #pragma unroll
-            for (int q = 0; q < kTileM / 32; ++q) {
-              const int row = row0 + q * 32 + lane;
+            for (int q = 0; q < kQ; ++q) {
+              const int row = row0 + (q0 + q) * 32 + lane;
               if (row < a.N) a.xn_out[(size_t)b * a.N + row] = xn2[q];
             }
           }
         }
         bool clamped = false;
 #pragma unroll
-        for (int q = 0; q < kTileM / 32; ++q) {
+        for (int q = 0; q < kQ; ++q) {
           alignas(16) T row[kExt];
           clamped |= ext_point_row<T, true>(xn2[q], row);
-          store_ext_row_sw32<T>(smem + L::kAExtOff + xb * kAExtBytes, q * 32 + lane, row);
+          store_ext_row_sw32<T>(smem + L::kAExtOff + xb * kAExtBytes, (q0 + q) * 32 + lane, row);
         }
         if (clamped) atomicCAS(a.err, DEV_OK, DEV_RANGE);
         // the norms for the epilogue's far-point check, once the epilogue has
@@ -504,27 +529,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // before tile g's norms are read
         if (!warp_wait(xnfree(xb), ((g >> 1) & 1) ^ 1, abort_flag, a.err, lane)) break;
 #pragma unroll
-        for (int q = 0; q < kTileM / 32; ++q) xnorm_s[xb * kTileM + q * 32 + lane] = xn2[q];
+        for (int q = 0; q < kQ; ++q) xnorm_s[xb * kTileM + (q0 + q) * 32 + lane] = xn2[q];
         fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
         __syncwarp();
         if (lane == 0) mbar_arrive(xnfull(xb));
       }
     }
-  } else if (warp == kLoadWarp) {
-    // ------------------------------------------------------------ point tiles
-    // (resident) tile g goes into the buffer of tile g - 2 as soon as that
-    // tile's MMAs are done, so it is requested a whole tile ahead of its use
-    if (RESIDENT && lane == 0) {
-      uint32_t g = 0;
-      for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++g) {
-        const int xb = g & 1;
-        if (!mbar_wait_spin(xempty(xb), ((g >> 1) & 1) ^ 1, abort_flag, a.err)) break;
-        mbar_arrive_expect_tx(xfull(xb), KB * kXBlockBytes);
-        const int b = tile / a.tiles_per_batch;
-        const int row0 = (tile % a.tiles_per_batch) * kTileM;
-        for (int kb = 0; kb < KB; ++kb)
-          tma_load_3d(&tmx, x_base + (xb * KB + kb) * kXBlockBytes, xfull(xb), kb * kBlockE, row0, b);
-      }
+    if (RESIDENT && warp == kLoadWarp && lane == 0) {
+      const uint32_t g = issued_tiles;
       // tail: the issued copies land (or are consumed) before exit
       const bool aborted = *abort_flag != 0;
       for (uint32_t gg = g > 2 ? g - 2 : 0; gg < g; ++gg)
@@ -630,20 +642,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         idx = bidx;
       }
       // combine the two column halves of each row: larger value, then lower
-      // index (one slot per row: the half-1 warps write a tile's slot a whole
-      // tile after the half-0 warps read the previous one)
+      // index (one slot per row; the two warps of a lane quadrant hand over
+      // through their own barriers, so each waits only for its partner, and
+      // the half-1 warp writes a tile's slot a whole tile after the half-0
+      // warp read the previous one)
       const uint32_t vpar = u & 1;
       float4 *slot = merge + r_in_tile;
       if (half == 1) {
-        if (!warp_wait(mempty(0), vpar ^ 1, abort_flag, a.err, lane)) { ok = false; break; }
+        if (!warp_wait(mempty(quad), vpar ^ 1, abort_flag, a.err, lane)) { ok = false; break; }
         *slot = make_float4(val, __int_as_float(idx), xn, 0.f);
         __syncwarp();
-        if (lane == 0) mbar_arrive(mfull(0));
+        if (lane == 0) mbar_arrive(mfull(quad));
       } else {
-        if (!warp_wait(mfull(0), vpar, abort_flag, a.err, lane)) { ok = false; break; }
+        if (!warp_wait(mfull(quad), vpar, abort_flag, a.err, lane)) { ok = false; break; }
         const float4 o = *slot;
         __syncwarp();
-        if (lane == 0) mbar_arrive(mempty(0));
+        if (lane == 0) mbar_arrive(mempty(quad));
         const float ov = o.x;
         const int oi = __float_as_int(o.y);
         if (ov > val || (ov == val && oi < idx)) {  // the value travels too: the keys compare it
