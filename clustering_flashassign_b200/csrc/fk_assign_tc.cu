@@ -25,9 +25,10 @@
 //               argmax per point.  Two warps share each TMEM lane quadrant
 //               and split the chunk's columns; their results are combined
 //               once per point tile,
-//   warp 10     (resident variant) ||x||^2 of each point tile from the shared
-//               copy, written as the tile's norm rows,
-//   warp 11     (resident variant) the point tiles (128 x d), one tile ahead.
+//   warps 10-11 (resident variant) ||x||^2 of each point tile (rows 0..63
+//               and 64..127), from the precomputed norms or the shared copy,
+//               written as the tile's norm rows; warp 11's lane 0 also
+//               requests the point tiles (128 x d), one tile ahead.
 // In the resident variant the MMA thread waits per chunk for its accumulator
 // (released by the epilogue) and for the stage, and commits once to the
 // stage's empty barrier: the stage is free and the epilogue may read the
