@@ -789,8 +789,11 @@ def run_baselines(args):
 def run_kernel_case(args):
     """Launch only one step kind on the bench workload (for profiler captures):
     assign = fk_assign, update = fk_update, lloyd = fk_lloyd with two
-    iterations (its assign uses the precomputed point norms and fills the
-    sort's tile histogram, as in the bench), each warmup + steps times."""
+    iterations, each warmup + steps times.  In an fk_lloyd call the first
+    assign sums the point norms from its shared tiles and stores them, the
+    second reads them; both fill the sort's tile histogram, as in the bench
+    (after the one fk_assign below, odd-numbered assign launches are first
+    assigns)."""
     import torch
 
     import clustering_flashassign_b200 as fk
