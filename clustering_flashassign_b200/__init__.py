@@ -37,7 +37,8 @@ FK_FAULT_NONE, FK_FAULT_ALLOC, FK_FAULT_H2D, FK_FAULT_LAUNCH = 0, 1, 2, 3
 
 DTYPES = {torch.float32: FK_F32, torch.float16: FK_F16, torch.bfloat16: FK_BF16}
 
-EXPORTS = ["fk_assign", "fk_update", "fk_sort", "fk_lloyd", "fk_assign_noalloc", "fk_status_string",
+EXPORTS = ["fk_assign", "fk_update", "fk_sort", "fk_lloyd", "fk_assign_noalloc", "fk_noalloc_device_error",
+           "fk_status_string",
            "fk_last_error", "fk_device_error", "fk_release", "fk_profile_enable", "fk_profile_read", "fk_profile_timeline",
            "fk_launch_count", "fk_version", "fk_selftest_bounded_wait", "fk_point_norms",
            "fk_init_centers", "fk_lloyd_step_partial", "fk_update_finalize", "fk_inject_fault"]
@@ -76,6 +77,7 @@ def _load():
         "fk_update": (I, [P, P, I, LL, I, I, P, P, P, I, P]),
         "fk_sort": (I, [P, I, LL, I, P, P, P, P]),
         "fk_assign_noalloc": (I, [P, P, I, LL, I, I, I, P, P]),
+        "fk_noalloc_device_error": (I, [P]),
         "fk_lloyd": (I, [ctypes.POINTER(FkShape), P, P, I, F, P, P, P, ctypes.POINTER(I),
                          ctypes.POINTER(FkOptions)]),
         "fk_status_string": (ctypes.c_char_p, [I]),
@@ -258,6 +260,11 @@ def fk_update_finalize(sums: torch.Tensor, counts: torch.Tensor, centers: torch.
 
 def fk_device_error(stream=None) -> int:
     return int(lib.fk_device_error(_stream(stream)))
+
+
+def fk_noalloc_device_error(stream=None) -> int:
+    """Status recorded by the fk_assign_noalloc kernels (read and cleared)."""
+    return int(lib.fk_noalloc_device_error(_stream(stream)))
 
 
 def fk_selftest_bounded_wait(limit_ns: int, stream=None) -> int:

@@ -72,3 +72,22 @@ extern "C" int fk_assign_noalloc(const void *x, const void *c, int B, long long 
   FK_TRY(launch_prep_cn(c, dtype, B, K, d, Kpad, cnx, err, s));
   return launch_assign_tc(x, c, cnx, nullptr, dtype, B, N, K, d, Kpad, ids, err, s);
 }
+
+// The error word sits in the static array, like the norm rows: read it with
+// blocking copies after the stream has drained, and clear it, allocating
+// nothing.
+extern "C" int fk_noalloc_device_error(fk_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float *base = nullptr;
+  FK_TRY(noalloc_base(&base));
+  FK_CUDA(cudaStreamSynchronize(s));
+  int h = DEV_OK;
+  FK_CUDA(cudaMemcpy(&h, base, sizeof(int), cudaMemcpyDeviceToHost));
+  if (h == DEV_OK) return FK_OK;
+  const int zero = DEV_OK;
+  FK_CUDA(cudaMemcpy(base, &zero, sizeof(int), cudaMemcpyHostToDevice));
+  if (h == DEV_TIMEOUT) return set_error(FK_ETIMEOUT, "a kernel's bounded wait expired");
+  if (h == DEV_RANGE)
+    return set_error(FK_EUNSUPPORTED, "a squared norm reached 2^32, beyond the fp16 tensor-core norm digits");
+  return set_error(FK_EINVAL, "unexpected device error code " + std::to_string(h));
+}

@@ -285,16 +285,29 @@ int fk_update_finalize(const float *sums, const int32_t *counts, int B, int K, i
  *   before any stream capture.
  *   All calls on a device share the array: calls that overlap on the GPU
  *   (e.g. on two streams) race and may return wrong ids.  The error word is
- *   cleared at the start of each call.  What the kernels record there is
- *   not reported by fk_device_error(), nor by this call (which does not
- *   synchronize): a bounded-wait timeout, and an fp16 squared norm of 2^32
- *   or more (a centroid or point with ||v|| >= 65536), where fk_assign
- *   reports FK_EUNSUPPORTED and this call returns unreliable ids.  Callers
- *   whose fp16 data may reach that range use fk_assign, or bf16 (whose norm
+ *   cleared at the start of each call.  What the kernels record there (a
+ *   bounded-wait timeout, or an fp16 squared norm of 2^32 or more: a
+ *   centroid or point with ||v|| >= 65536, where the ids are unreliable) is
+ *   not reported by this call, which does not synchronize, nor by
+ *   fk_device_error(): read it with fk_noalloc_device_error().  Callers
+ *   whose fp16 data may reach that range can also use bf16 (whose norm
  *   digits have the fp32 range).
  */
 int fk_assign_noalloc(const void *x, const void *c, int B, long long N, int K, int d, int dtype,
                       int32_t *ids, fk_stream_t stream);
+
+/*
+ * fk_noalloc_device_error -- the error word of fk_assign_noalloc's static
+ * scratch on the current device (an interface addition, like that call).
+ * Synchronizes `stream`, reads the word and clears it with blocking copies;
+ * allocates nothing.  It reports what the fk_assign_noalloc calls since the
+ * last clear recorded (each call also clears the word when it starts), so
+ * call it after the call whose result matters, with no other such call in
+ * flight on the device.  Returns FK_OK, FK_ETIMEOUT (a bounded wait in a
+ * kernel gave up) or FK_EUNSUPPORTED (an fp16 squared norm of 2^32 or
+ * more: that call's ids are unreliable).
+ */
+int fk_noalloc_device_error(fk_stream_t stream);
 
 /* Static text for a status code. */
 const char *fk_status_string(int status);
@@ -305,7 +318,9 @@ const char *fk_last_error(void);
 /*
  * Synchronizes `stream`, reads and clears the device error word of its
  * workspace.  Returns FK_OK, FK_ETIMEOUT (a bounded wait in a kernel gave
- * up) or FK_EINVAL (an id outside [0, K) reached fk_update / fk_sort).
+ * up), FK_EUNSUPPORTED (an fp16 squared norm of 2^32 or more reached the
+ * tensor-core assign's norm digits) or FK_EINVAL (an id outside [0, K)
+ * reached fk_update / fk_sort).
  */
 int fk_device_error(fk_stream_t stream);
 

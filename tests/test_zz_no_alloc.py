@@ -89,3 +89,28 @@ def test_noalloc_fp32_on_cuda_cores_matches_the_oracle_where_fk_assign_uses_tf32
         tc = torch.empty((B, N), dtype=torch.int32, device="cuda")
         fk.fk_assign(x, c, tc)
         check_ids(tc.cpu().numpy(), xn, "f32", chat, ref, gap)
+
+
+def test_noalloc_reports_a_norm_beyond_the_fp16_digit_range():
+    """What the kernels record in the static error word is read (and cleared)
+    by fk_noalloc_device_error, which allocates nothing either."""
+    import clustering_flashassign_b200 as fk
+    B, N, K, d = 1, 300, 40, 128
+    x, c = _inputs(B, N, K, d, "f16", 9)
+    assert fk.fk_noalloc_device_error() == fk.FK_OK
+    c[0, 5] = 6000.0   # ||c||^2 = 128 * 3.6e7 = 4.6e9 > 2^32
+    got = torch.full((B, N), -1, dtype=torch.int32, device="cuda")
+    assert _raw_noalloc(fk, x, c, got) == fk.FK_OK   # asynchronous: nothing read yet
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    assert fk.fk_noalloc_device_error() == fk.FK_EUNSUPPORTED
+    assert "2^32" in fk.fk_last_error()
+    assert fk.fk_noalloc_device_error() == fk.FK_OK   # cleared
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, "fk_noalloc_device_error changed free device memory"
+    c[0, 5] = 4000.0   # ||c||^2 = 2.05e9 < 2^32: fine
+    ref = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    fk.fk_assign(x, c, ref)
+    assert _raw_noalloc(fk, x, c, got) == fk.FK_OK
+    assert fk.fk_noalloc_device_error() == fk.FK_OK
+    assert torch.equal(got, ref)
