@@ -32,9 +32,8 @@
 // In the resident variant the MMA thread waits per chunk for its accumulator
 // (released by the epilogue) and for the stage, and commits once to the
 // stage's empty barrier: the stage is free and the epilogue may read the
-// accumulator.  With two K-blocks it also commits after K-block 0, so the
-// producer refills that half of the stage half a chunk earlier; the producer
-// waits for nothing else and runs ahead as far as the stages allow.  The
+// accumulator; the producer waits for nothing else and runs ahead as far as
+// the stages allow.  The
 // centroids' norm rows are stored pre-swizzled (fk_centroids.cu) and arrive
 // by one bulk copy per chunk: the TMA unit moves tiles row by row, and 256
 // rows of 32 bytes cost it about as much as 256 rows of 128 bytes.
@@ -153,8 +152,8 @@ struct Layout {
   static constexpr uint32_t kBarOff = kStagesOff + STAGES * kStageBytes;
   // barriers: full[S], empty[S], efull[E], eempty[E], xfull[2], xempty[2],
   //           xnfull[2], accfull[2], accempty[2], mfull[4], mempty[4], drain,
-  //           xnfree[2], kbfree[S]
-  static constexpr int kNumBars = 3 * STAGES + 2 * kExtSlots + 21;
+  //           xnfree[2]
+  static constexpr int kNumBars = 2 * STAGES + 2 * kExtSlots + 21;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag
   static constexpr uint32_t kMergeOff = (kMiscOff + 16 + 15) / 16 * 16;
   // resident: ||x||^2 of the rows of the two point-tile buffers, for the
@@ -217,7 +216,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto mempty = [&](int q) { return bar0 + 8u * (kB2 + 14 + q); };
   const uint32_t drain = bar0 + 8u * (kB2 + 18);
   auto xnfree = [&](int i) { return bar0 + 8u * (kB2 + 19 + i); };
-  auto kbfree = [&](int s) { return bar0 + 8u * (kB2 + 21 + s); };
   float *xnorm_s = reinterpret_cast<float *>(smem + L::kXnOff);  // [2][kTileM], resident only
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
@@ -229,7 +227,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
-      mbar_init(kbfree(s), 1);  // resident, two K-blocks: K-block 0 of the stage read
     }
     for (int e = 0; e < kExtSlots; ++e) {
       mbar_init(efull(e), 1);
@@ -303,29 +300,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = chunk_lo(task); ok && c < chunk_hi(task); ++c) {
           if (RESIDENT) {  // the whole chunk and its norm rows in one stage
             // empty(s) is committed once per chunk by the MMA thread: the
-            // stage is free and the epilogue may read the chunk's accumulator.
-            // With two K-blocks, K-block 0 is refilled as soon as the chunk
-            // STAGES back has read it (kbfree), half a chunk earlier; its
-            // bytes are expected before the copy and the one arrival comes
-            // with the rest, so the phase cannot complete early.
+            // stage is free and the epilogue may read the chunk's accumulator
             const int s = f % STAGES;
-            const uint32_t par = ((f / STAGES) & 1) ^ 1;
+            if (!mbar_wait_spin(empty(s), ((f / STAGES) & 1) ^ 1, abort_flag, a.err)) { ok = false; break; }
             const uint32_t dst = st_base + s * L::kStageBytes;
-            if constexpr (KB == 2) {
-              if (!mbar_wait_spin(kbfree(s), par, abort_flag, a.err)) { ok = false; break; }
-              mbar_expect_tx(full(s), kCBlockBytes);
-              tma_load_3d(&tmc, dst, full(s), 0, c * kChunkN, b);
-            }
-            if (!mbar_wait_spin(empty(s), par, abort_flag, a.err)) {
-              if (KB == 2) {  // let the phase complete as K-block 0 lands; the tail drains it
-                mbar_arrive(full(s));
-                ++f;
-              }
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(full(s), L::kStageBytes - (KB == 2 ? kCBlockBytes : 0u));
-            for (int kb = KB == 2 ? 1 : 0; kb < KB; ++kb)
+            mbar_arrive_expect_tx(full(s), L::kStageBytes);
+            for (int kb = 0; kb < KB; ++kb)
               tma_load_3d(&tmc, dst + kb * kCBlockBytes, full(s), kb * kBlockE, c * kChunkN, b);
             bulk_load(dst + KB * kCBlockBytes, a.cnx + ((size_t)b * a.nchunks + c) * kBExtBytes, kBExtBytes,
                       full(s));
@@ -391,7 +371,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int k = 0; k < kBlockK / 16; ++k)
                 mma_t<T>(d_tmem, desc_k_sw128(a_addr + k * 32), desc_k_sw128(b_addr + k * 32), a.idesc,
                         (kb | k) != 0 ? 1u : 0u);
-              if (KB == 2 && kb == 0) mma_commit(kbfree(s));  // K-block 0 may be refilled
             }
             // the norm step: acc += A_ext . B_ext (fk_norms.cuh)
             mma_t<T>(d_tmem, desc_k_sw32(a_ext), desc_k_sw32(stage + KB * kCBlockBytes), a.idesc, 1u);
